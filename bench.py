@@ -1,0 +1,393 @@
+"""Batch-1 decode benchmark of the 7B-shape INT4 weight-only decoder on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl i4|reference]
+
+A step is one decode token: one replay of the captured CUDA graph (28 layers x
+{qkv+RoPE+KV append, paged attention, o, RMSNorm+gate/up+SiLU, down} + final
+norm, lm_head and argmax: 141 kernels). Setup (untimed): random-init INT4
+weights (seed 0), a 512-token prompt of uniform random ids fed through the
+same graph, then W warm-up tokens; then K timed tokens, each at a context one
+longer than the last. Every token streams 3.65 GB of INT4 weights and scales
+(more than the 126 MB L2), so no L2 flush is needed between steps.
+
+Printed (rank 0, one JSON line): tok/s over all ranks (replicas: one sequence
+per GPU, no exchange), ms/token (max over ranks, CUDA events), the end-to-end
+rate through the public API with the token copied host->device and the next
+token device->host every step, the roofline of the dominant kernel (the
+RMSNorm+gate/up+SiLU GEMV) against the measured HBM copy bandwidth, the whole
+step against 8 TB/s and the measured bandwidth, SM clocks sampled during the
+timed region, and the CPU oracle timed on a bounded sample.
+
+--impl reference times the CPU oracle instead (rank 0 only), each step one
+decoder layer of one token at context 513, scaled to tok/s.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tok/s at batch 1 (7B-shape INT4); INT4 GEMV HBM GB/s vs B200 peak"
+WORKLOAD = ("qwen2.5-7b-shape decoder (28 layers, hidden 3584, mlp 18944, 28q/4kv heads, head_dim 128, "
+            "vocab 152064), int4 group-128 fp16-scale weights, batch 1, 512-token prompt then greedy decode, "
+            "paged KV page 16, one CUDA graph per token")
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id, self.proc, self.lines = gpu_id, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", self.gpu_id], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        if not self.lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except Exception:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_from_profile(kernel_src: str):
+    """DRAM bytes per launch of the gate/up GEMV from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "gemv_gate_up_qwen7b.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    src_hash = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256_16") != src_hash:
+        return None
+    try:
+        return float(vals["dram_bytes_per_full_launch"])
+    except Exception:
+        return None
+
+
+def oracle_cpu_sample(shape, layers_np, glob_np, n_tokens: int = 2):
+    """The CPU oracle as it stands: n_tokens decode steps at position 512 with the KV
+    cache below it filled with random fp16 values."""
+    import numpy as np
+
+    import oracle
+    from int4_weight_only_02_b200 import synth
+    dec = oracle.DecoderOracle(shape, layers_np, glob_np, synth.page_table(shape, 0), num_pages=shape.max_pages)
+    rng = np.random.default_rng(123)
+    used = (512 + n_tokens + shape.page_size - 1) // shape.page_size
+    for li in range(shape.layers):
+        for pool in (dec.k_pools[li], dec.v_pools[li]):
+            for p in dec.page_table[:used]:
+                pool[p] = (rng.standard_normal(pool[p].shape) * 4).astype(np.float16)
+    t0 = time.perf_counter()
+    tok = 1
+    for i in range(n_tokens):
+        logits, _ = dec.forward([tok], 512 + i)
+        tok = oracle.argmax(logits)
+    el = time.perf_counter() - t0
+    return {"value": round(n_tokens / el, 4), "unit": "tok/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{n_tokens} full decode tokens (28 layers + lm_head) at positions 512..{511 + n_tokens}, "
+                      f"KV below filled with random fp16, fp64 C/numpy oracle on all host cores "
+                      f"({el:.1f} s)"}
+
+
+def run_reference(args):
+    """CPU oracle arm: each step is one decoder layer of one token at context 513."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    import numpy as np
+
+    import oracle
+    from int4_weight_only_02_b200 import synth
+    shape = synth.QWEN7B
+    one = synth.ModelShape(layers=1)
+    lw = [synth.layer_weights(shape, 0, 0)]
+    glob = synth.global_weights(shape, 0)
+    dec = oracle.DecoderOracle(one, lw, glob, synth.page_table(shape, 0), num_pages=shape.max_pages)
+    rng = np.random.default_rng(5)
+    for pool in (dec.k_pools[0], dec.v_pools[0]):
+        for p in dec.page_table[:33]:
+            pool[p] = (rng.standard_normal(pool[p].shape) * 4).astype(np.float16)
+    r = glob["embed"][[7]].astype(np.float16)
+    t0 = time.perf_counter()
+    x = oracle.rmsnorm(r[-1], glob["ln_final"], shape.eps)
+    oracle.int4_gemv(glob["w_lm"], glob["s_lm"], x, None, shape.group, np.float32)
+    t_lm = time.perf_counter() - t0
+    for _ in range(args.warmup):
+        dec.layer(0, r, [512])
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        dec.layer(0, r, [512])
+        times.append(time.perf_counter() - t0)
+    t_layer = statistics.mean(times)
+    ms_tok = (shape.layers * t_layer + t_lm) * 1e3
+    value = 1e3 / ms_tok
+    sample = (f"each step = one decoder layer of one token at context 513 (fp64 oracle, {os.cpu_count()} host "
+              f"cores); tok/s = 1 / (28 x mean layer time + lm_head time {t_lm * 1e3:.0f} ms)")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "tok/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_tok, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "prompt": 512},
+            "cpu_baseline": {"value": round(value, 5), "unit": "tok/s", "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=128)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="i4", choices=["i4", "reference"])
+    ap.add_argument("--prompt", type=int, default=512)
+    ap.add_argument("--eager-steps", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pdl", type=int, default=None, help="override programmatic dependent launch (0/1)")
+    ap.add_argument("--unpack", type=int, default=None, help="override the GEMV unpack variant (0/1)")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import int4_weight_only_02_b200 as i4
+    from int4_weight_only_02_b200 import synth
+    from int4_weight_only_02_b200.runtime import to_device
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    i4.lib()
+    if args.pdl is not None:
+        i4.set_option("pdl", args.pdl)
+    if args.unpack is not None:
+        i4.set_option("unpack", args.unpack)
+
+    shape = synth.QWEN7B
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    layers_np = []
+    model = i4.DeviceModel.__new__(i4.DeviceModel)
+    model.shape, model.device, model.layers = shape, dev, []
+    for li in range(shape.layers):
+        lw = synth.layer_weights(shape, li, 0)
+        model.layers.append({k: to_device(v, dev) for k, v in lw.items()})
+        if want_cpu:
+            layers_np.append(lw)
+    glob_np = synth.global_weights(shape, 0)
+    model.glob = {k: to_device(v, dev) for k, v in glob_np.items()}
+    if not want_cpu:
+        glob_np = None
+
+    prompt = synth.prompt_tokens(shape, args.prompt, seed=rank)
+    seq = i4.Sequence(model, synth.page_table(shape, 0), prompt)
+    graph = i4.DecodeGraph(model, seq)
+    n_k = graph.kernel_count
+    stream = torch.cuda.current_stream()
+
+    # prompt ingestion and warm-up (untimed)
+    for _ in range(args.prompt + args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    ctx0 = int(seq.ctx_len.item())
+
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_id) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_tok = ms_max / args.steps
+    status = int(seq.status.item())
+    ctx1 = int(seq.ctx_len.item())
+
+    # end to end through the public API: token host->device, step, next token device->host, every step
+    tok_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
+    out_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
+    tok_h.copy_(seq.token.cpu())
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        seq.token.copy_(tok_h, non_blocking=True)
+        graph.replay()
+        out_h.copy_(seq.token, non_blocking=True)
+        stream.synchronize()
+        tok_h[0] = out_h[0]
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_tok_s = world * args.steps / (float(t.item()) / 1e3)
+
+    # eager launches of the same kernels (the pages' eager-vs-graph comparison)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.eager_steps):
+        graph.eager()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    eager_ms = e0.elapsed_time(e1) / max(args.eager_steps, 1)
+
+    # dominant kernel alone: RMSNorm + gate/up GEMV + SiLU of each layer (70 MB each, L2-cold)
+    def time_kernel(index_fn, reps=2):
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(shape.layers * reps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(shape.layers * reps)]
+        for r in range(reps):
+            for li in range(shape.layers):
+                j = r * shape.layers + li
+                starts[j].record(stream)
+                graph.launch_kernel(index_fn(li))
+                ends[j].record(stream)
+        torch.cuda.synchronize()
+        d = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        return statistics.mean(d[shape.layers:]) if reps > 1 else statistics.mean(d)
+
+    h, inter = shape.hidden, shape.inter
+    gu_bytes = 2 * inter * (h // 2) + 2 * inter * (h // 128) * 2 + 2 * h * 2 + inter * 2
+    gu_ms = time_kernel(lambda li: 5 * li + 3)
+    down_bytes = h * (inter // 2) + h * (inter // 128) * 2 + inter * 2 + 2 * h * 2
+    down_ms = time_kernel(lambda li: 5 * li + 4)
+    qkv_rows = shape.qkv_rows
+    qkv_bytes = qkv_rows * (h // 2) + qkv_rows * (h // 128) * 2 + 2 * qkv_rows * 2 + 2 * h * 2
+    qkv_ms = time_kernel(lambda li: 5 * li + 0)
+    o_bytes = h * (h // 2) + h * (h // 128) * 2 + h * 2 + 2 * h * 2
+    o_ms = time_kernel(lambda li: 5 * li + 2)
+    torch.cuda.synchronize()
+    # restore a consistent residual/KV state is not needed afterwards: nothing else runs
+
+    peak, peak_kind = measured_peaks()
+    gu_gbs = gu_bytes / (gu_ms * 1e-3) / 1e9
+    traffic = traffic_from_profile(os.path.join(ROOT, "int4_weight_only_02_b200", "csrc", "gemv.cu"))
+
+    weight_bytes = model.weight_bytes()
+    ctx_mean = (ctx0 + ctx1 - 1) / 2.0
+    kv_bytes = 2 * shape.layers * shape.n_kv * shape.head_dim * 2 * ctx_mean
+    step_bytes = weight_bytes + kv_bytes
+    step_gbs = step_bytes / (ms_tok * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": round(world * args.steps / (ms_max / 1e3), 2), "unit": "tok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_tok, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "prompt": args.prompt, "ctx_first": ctx0, "ctx_last": ctx1 - 1,
+                   "arith": "int4 weights x fp16 activations, fp32 accumulate", "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2: 3.65 GB of weights streamed per step, no flush",
+                   "kernels_per_step": n_k, "status": status},
+        "roofline": {"kernel": "rmsnorm+gate/up int4 gemv+silu (K=3584, N=37888)", "bound": "hbm",
+                     "achieved": round(gu_gbs, 1), "peak": peak, "peak_kind": f"{peak_kind} copy bandwidth",
+                     "unit": "GB/s", "frac": round(gu_gbs / peak, 4), "traffic": traffic,
+                     "bytes_per_launch": gu_bytes, "us_per_launch": round(gu_ms * 1e3, 2)},
+        "kernels": {
+            "qkv": {"us": round(qkv_ms * 1e3, 2), "GBs": round(qkv_bytes / (qkv_ms * 1e-3) / 1e9, 1)},
+            "o": {"us": round(o_ms * 1e3, 2), "GBs": round(o_bytes / (o_ms * 1e-3) / 1e9, 1)},
+            "gate_up": {"us": round(gu_ms * 1e3, 2), "GBs": round(gu_gbs, 1)},
+            "down": {"us": round(down_ms * 1e3, 2), "GBs": round(down_bytes / (down_ms * 1e-3) / 1e9, 1)}},
+        "step_roofline": {"bytes_per_step": int(step_bytes), "achieved_GBs": round(step_gbs, 1),
+                          "frac_of_8TBs": round(step_gbs / NOMINAL_HBM_GBS, 4),
+                          "frac_of_measured": round(step_gbs / peak, 4)},
+        "eager_ms_per_step": round(eager_ms, 3),
+        "e2e": {"value": round(e2e_tok_s, 2), "unit": "tok/s", "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4},
+        "gpu_launches": args.steps * n_k,
+        "clocks": clocks.summary(),
+    }
+    graph.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if want_cpu:
+            del model, seq
+            line["cpu_baseline"] = oracle_cpu_sample(shape, layers_np, glob_np)
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,260 @@
+/*
+ * i4rt -- batch-1 INT4 weight-only decode of a Qwen2.5-7B-shaped decoder on
+ * NVIDIA B200 (sm_100a). C ABI of libi4rt.so.
+ *
+ * The operations follow "How To Build Your Own LLM Runtime From Scratch"
+ * ("Technical Details": INT4 weight packing and dequantisation, a paged KV
+ * cache, attention over it, and a decode step captured as one CUDA graph; the
+ * CUDA-graph item of the same section gives eager ~119 ms/token versus graph
+ * replay ~17 ms/token on H100). The pages fix no formats; this library uses:
+ *
+ *   INT4 weights  w[N][K/8] uint32. Word j of row n holds k = 8j .. 8j+7;
+ *                 field i (bits 4i..4i+3) is k = 8j+i as a two's-complement
+ *                 integer in [-8, 7].
+ *   scales        s[N][K/group] fp16, symmetric: W[n][k] = q[n][k] * s[n][k/group].
+ *   fp16          IEEE binary16, passed as uint16_t bit patterns.
+ *   KV pools      [num_pages][n_kv][page_size][head_dim] fp16, one K and one V
+ *                 pool per layer; token t of sequence b is in page
+ *                 page_table[b][t / page_size], slot t % page_size.
+ *
+ * Conventions shared by every call:
+ *   - Return value: I4_OK (0) or a negative I4_E* status. i4_last_error()
+ *     returns a text for the last failure on the calling thread.
+ *   - Tensor pointers are device memory owned by the caller unless a comment
+ *     says "host". The library never frees caller memory.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *     asynchronous on it; arguments are validated on the host before any
+ *     launch, and an invalid call launches nothing.
+ *   - No call allocates device memory, synchronises the device or reads
+ *     device memory on the host, except decode_step_graph_create/destroy.
+ */
+#ifndef I4RT_H
+#define I4RT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define I4_API __attribute__((visibility("default")))
+#else
+#define I4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define I4_OK 0
+#define I4_EINVAL (-1)       /* null pointer, bad shape or size */
+#define I4_EALIGN (-2)       /* pointer alignment below the stated requirement */
+#define I4_EUNSUPPORTED (-3) /* valid but not implemented (e.g. head_dim != 128) */
+#define I4_ECUDA (-4)        /* a CUDA runtime call or launch failed */
+#define I4_ENOMEM (-5)       /* device allocation failed (graph create only) */
+
+/* Text of the last failure on this thread ("" if none). Never NULL. */
+I4_API const char *i4_last_error(void);
+
+/* Library version string. */
+I4_API const char *i4_version(void);
+
+/*
+ * INT4 weight-only linear layer ("INT4 dequantization" fused into the product):
+ *   y[m][n] = sum_k q[n][k] * s[n][k/group] * x[m][k]  (+ bias[n])
+ * accumulated in fp32, stored as fp16 (y_is_fp32 = 0) or fp32 (y_is_fp32 = 1).
+ *   w      [N][K/8] uint32, 16-byte aligned;
+ *   scales [N][K/group] fp16, 2-byte aligned;
+ *   x      [M][K] fp16, 16-byte aligned;  bias [N] fp16 or NULL;
+ *   y      [M][N], 4-byte aligned for fp32.
+ * Requires group == 128, K % 128 == 0, K <= 32768, 1 <= M <= 8, N >= 1.
+ */
+I4_API int int4_gemv(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
+              int y_is_fp32, int M, int N, int K, int group, void *stream);
+
+/*
+ * Test export: q[n][k] = signed field of w (bit-exact unpack check).
+ *   w [N][K/8] uint32; q [N][K] int8. K % 8 == 0.
+ */
+I4_API int i4_int4_unpack(const uint32_t *w, int8_t *q, int N, int K, void *stream);
+
+/*
+ * Paged grouped-query decode attention ("paged KV cache, and attention"; the
+ * softmax must be exact at partially filled last pages). For each sequence b
+ * and query head h, with kv head g = h / (Hq / Hkv) and n = ctx_len[b]:
+ *   s_t = scale * q[b][h] . K[g][t],  p = softmax(s over t < n),
+ *   out[b][h] = sum_t p_t V[g][t]        (fp32 math, fp16 out)
+ * computed as split-K over pages with a log-sum-exp merge.
+ *   q, out      [B][Hq][D] fp16, 16-byte aligned;
+ *   k_pool, v_pool [num_pages][Hkv][page_size][D] fp16, 16-byte aligned;
+ *   page_table  [B][max_pages_per_seq] int32 physical page ids;
+ *   ctx_len     [B] int32 device array, tokens per sequence INCLUDING the
+ *               current one, 1 <= ctx_len[b] <= max_pages_per_seq * page_size;
+ *   ws          workspace of paged_gqa_decode_ws_bytes(...) bytes, 256-byte
+ *               aligned, ZEROED by the caller before its first use; every call
+ *               leaves its counters zero again. Calls sharing one ws must not
+ *               overlap on the GPU.
+ * Requires D == 128, 1 <= Hq / Hkv <= 8 (Hq % Hkv == 0), page_size a power of
+ * two in [8, 256], B >= 1.
+ */
+I4_API size_t paged_gqa_decode_ws_bytes(int B, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq);
+I4_API int paged_gqa_decode(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_pool, const int32_t *page_table,
+                     const int32_t *ctx_len, uint16_t *out, int B, int Hq, int Hkv, int D, int page_size,
+                     int max_pages_per_seq, float scale, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Test export: out[b][g][t][:] = pool row of token t (t < ctx_len[b]) for kv
+ * head g, in token order (bit-exact page-indexing check). Rows t >= ctx_len[b]
+ * are left untouched.  out [B][Hkv][max_ctx][D] fp16.
+ */
+I4_API int i4_paged_gather(const uint16_t *pool, const int32_t *page_table, const int32_t *ctx_len, uint16_t *out, int B,
+                    int Hkv, int D, int page_size, int max_pages_per_seq, int max_ctx, void *stream);
+
+/*
+ * RMSNorm and RoPE + KV append, the glue of a decoder layer. Either part may
+ * be skipped by leaving its first pointer NULL; when both are given the norm
+ * runs first.
+ *
+ * Norm part (x_in != NULL), for each of M rows of H values:
+ *   if resid != NULL:  resid = fp16(resid + x_in), v = resid  else v = x_in
+ *   out = fp16(v / sqrt(mean(v^2) + eps) * gamma)          (fp32 math)
+ *   x_in, resid, out [M][H] fp16; gamma [H] fp16; H % 8 == 0, H <= 32768.
+ *
+ * RoPE part (qkv != NULL), for each of B sequences at position pos[b]:
+ *   qkv [B][(Hq + 2 Hkv) * D] fp16 laid out [q heads | k heads | v heads];
+ *   q and k heads are rotated in place (rotate-half pairs (i, i + D/2),
+ *   angle pos * theta^(-2i/D), fp32 math), then k and v of each kv head are
+ *   written to page_table[b][pos / page_size], slot pos % page_size of the
+ *   pools (skipped when k_pool is NULL). D == 128.
+ */
+typedef struct i4_rmsnorm_rope_args {
+    /* norm part */
+    const uint16_t *x_in;
+    uint16_t *resid;
+    const uint16_t *gamma;
+    uint16_t *out;
+    int M, H;
+    float eps;
+    /* rope + append part */
+    uint16_t *qkv;
+    const int32_t *pos;
+    int B, Hq, Hkv, D;
+    float theta;
+    uint16_t *k_pool, *v_pool;
+    const int32_t *page_table;
+    int page_size, max_pages_per_seq;
+} i4_rmsnorm_rope_args;
+
+I4_API int rmsnorm_rope(const i4_rmsnorm_rope_args *args, void *stream);
+I4_API int i4_rmsnorm(const uint16_t *x_in, uint16_t *resid, const uint16_t *gamma, uint16_t *out, int M, int H, float eps,
+               void *stream);
+I4_API int i4_rope_kv_append(uint16_t *qkv, const int32_t *pos, int B, int Hq, int Hkv, int D, float theta,
+                      uint16_t *k_pool, uint16_t *v_pool, const int32_t *page_table, int page_size,
+                      int max_pages_per_seq, void *stream);
+
+/*
+ * SwiGLU gate: out[m][i] = fp16(silu(g) * u), g = gate_up[m][i], u = gate_up[m][I + i],
+ * silu(g) = g / (1 + exp(-g)) in fp32.  gate_up [M][2I] fp16; out [M][I] fp16.
+ */
+I4_API int silu_mul(const uint16_t *gate_up, uint16_t *out, int M, int I, void *stream);
+
+/* ---------------------------------------------------------------- decode step */
+
+typedef struct i4_model_desc {
+    int n_layers, hidden, intermediate, n_q_heads, n_kv_heads, head_dim, vocab;
+    int group;      /* INT4 group size along K, must be 128 */
+    int page_size;  /* tokens per KV page */
+    int max_ctx;    /* page table length * page_size */
+    float rope_theta, rms_eps;
+} i4_model_desc;
+
+typedef struct i4_layer_weights {
+    const uint32_t *w_qkv;     /* [(Hq + 2 Hkv) D][hidden/8], rows [q | k | v] */
+    const uint16_t *s_qkv;     /* [(Hq + 2 Hkv) D][hidden/128] */
+    const uint16_t *b_qkv;     /* [(Hq + 2 Hkv) D] */
+    const uint32_t *w_o;       /* [hidden][Hq D/8] */
+    const uint16_t *s_o;
+    const uint32_t *w_gate_up; /* [2 intermediate][hidden/8], rows [gate | up] */
+    const uint16_t *s_gate_up;
+    const uint32_t *w_down;    /* [hidden][intermediate/8] */
+    const uint16_t *s_down;
+    const uint16_t *ln_in;     /* input_layernorm gamma [hidden] */
+    const uint16_t *ln_post;   /* post_attention_layernorm gamma [hidden] */
+} i4_layer_weights;
+
+typedef struct i4_model_weights {
+    const uint16_t *embed;             /* [vocab][hidden] fp16 */
+    const i4_layer_weights *layers;    /* HOST array of n_layers (copied at create) */
+    const uint16_t *ln_final;          /* [hidden] */
+    const uint32_t *w_lm;              /* [vocab][hidden/8] */
+    const uint16_t *s_lm;              /* [vocab][hidden/128] */
+} i4_model_weights;
+
+/*
+ * One sequence's decode state, all device memory owned by the caller.
+ * A step reads token[0] at position pos[0] (ctx_len[0] must equal pos[0] + 1),
+ * appends its K/V, writes fp32 logits [vocab], and then advances the state on
+ * the device: pos += 1, ctx_len += 1, token = prompt[pos] while pos < n_prompt,
+ * else the argmax of the logits (lowest index on ties); history[pos] = token.
+ * Steps whose position would reach max_ctx set *status to 1 and do nothing.
+ */
+typedef struct i4_seq_state {
+    int32_t *token, *pos, *ctx_len;   /* [1] each */
+    const int32_t *page_table;        /* [max_ctx / page_size] */
+    uint16_t *const *k_pools;         /* HOST array of n_layers device pointers */
+    uint16_t *const *v_pools;         /* HOST array of n_layers device pointers */
+    int num_pages;                    /* pages in each pool */
+    float *logits;                    /* [vocab] */
+    const int32_t *prompt;            /* [n_prompt] or NULL */
+    int n_prompt;
+    int32_t *history;                 /* [max_ctx] or NULL */
+    int32_t *status;                  /* [1], 0 = ok */
+} i4_seq_state;
+
+typedef struct i4_graph i4_graph;
+
+/*
+ * Build the decode step: allocates its private workspace, validates shapes and
+ * captures every kernel of one token into a CUDA graph on an internal stream.
+ * The descriptors are copied; the device buffers they point at must outlive
+ * the graph. Returns I4_ENOMEM, I4_EINVAL, I4_EUNSUPPORTED or I4_ECUDA on failure.
+ */
+I4_API int decode_step_graph_create(const i4_model_desc *desc, const i4_model_weights *weights, const i4_seq_state *seq,
+                             i4_graph **out);
+/* Launch the captured token step on `stream` (one cudaGraphLaunch). */
+I4_API int decode_step_graph_replay(i4_graph *g, void *stream);
+/* The same step as individual kernel launches on `stream` (no graph). */
+I4_API int decode_step_eager(i4_graph *g, void *stream);
+/* Kernel launches in one step (eager or inside the graph). */
+I4_API int decode_step_kernel_count(const i4_graph *g);
+I4_API int decode_step_graph_destroy(i4_graph *g);
+/*
+ * Benchmark export: launch only kernel `index` (0 <= index < kernel count) of
+ * the step on `stream`, with the step's arguments. Per layer l the kernels are
+ * 5l+0 qkv, 5l+1 attention, 5l+2 o, 5l+3 gate/up, 5l+4 down; the last is
+ * lm_head + argmax, which advances the sequence state. Kernels that add into
+ * the residual or write K/V leave values that the next full step rewrites.
+ */
+I4_API int decode_step_launch_kernel(i4_graph *g, int index, void *stream);
+
+/*
+ * Library options, applied to graphs created afterwards and to later calls:
+ *   "pdl"    0/1: launch the kernels of a decode step with programmatic
+ *            dependent launch (each kernel still waits for its predecessor's
+ *            results before reading them);
+ *   "unpack" 0/1: INT4 unpack variant of the GEMV (0 exact fp16 values,
+ *            1 offset-binary fp16 subnormals with a per-chunk sum(x) correction).
+ * Not thread-safe; set options before creating graphs.
+ */
+I4_API int i4_set_option(const char *name, int value);
+
+/*
+ * int4_gemv with an explicit unpack variant (0 or 1, as above) and a cap on the
+ * number of CTAs (0 = none); for tests and benchmarks.
+ */
+I4_API int i4_int4_gemv_variant(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
+                         int y_is_fp32, int M, int N, int K, int unpack, int max_ctas, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* I4RT_H */

@@ -1,0 +1,27 @@
+// Internal interface of the paged decode attention kernel (see attention.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace i4 {
+
+struct AttnParams {
+    const uint16_t *q, *k_pool, *v_pool;
+    const int32_t *page_table, *ctx_len;
+    uint16_t *out;
+    int B, Hq, Hkv, page_size, max_pages, splits;
+    float scale;
+    char *ws;
+    size_t counters_off, ml_off, acc_off;
+};
+
+struct AttnWs {
+    int splits;
+    size_t counters_off, ml_off, acc_off, bytes;
+};
+
+int attn_splits(int B, int Hkv, int page_size, int max_pages);
+AttnWs attn_ws_layout(int B, int Hq, int Hkv, int page_size, int max_pages);
+int launch_paged_gqa_decode(const AttnParams &p, cudaStream_t stream, bool pdl);
+
+}  // namespace i4

@@ -1,0 +1,361 @@
+// The decode step of the 28-layer decoder as one captured CUDA graph.
+//
+// "How To Build Your Own LLM Runtime From Scratch" ("Technical Details", CUDA
+// graph item; second lesson): per-launch driver overhead dominated their eager
+// decode (~119 ms/token) and graph replay removed it (~17 ms/token on H100)
+// without changing a kernel. Here one token is 5 kernels per layer plus one:
+//
+//   qkv   : RMSNorm(r) (layer 0: embedding gather) -> INT4 GEMV -> +bias, RoPE, K/V append
+//   attn  : paged GQA decode attention (split-K + LSE merge)
+//   o     : INT4 GEMV -> r += fp16(y)
+//   gu    : RMSNorm(r) -> INT4 GEMV [gate | up] -> SiLU(gate) * up
+//   down  : INT4 GEMV -> r += fp16(y)
+//   lm    : RMSNorm(r) -> INT4 GEMV (fp32 logits) -> argmax -> token, pos, ctx_len advance
+//
+// All per-token state (token, position, context length) lives in device
+// memory and is advanced by the last kernel, so the same graph is replayed for
+// every token with no host work in between. Kernels may be launched with
+// programmatic dependent launch; each one waits (griddepcontrol.wait) before
+// reading what its predecessors wrote.
+#include <cmath>
+#include <string>
+#include <vector>
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemv.cuh"
+
+namespace i4 {
+int launch_rope_table(float2 *cs, int max_ctx, int d, double theta, cudaStream_t stream);
+bool g_dry_run = false;
+bool g_pdl = false;
+}  // namespace i4
+
+using namespace i4;
+
+struct i4_graph {
+    i4_model_desc d;
+    i4_model_weights w;
+    std::vector<i4_layer_weights> layers;
+    i4_seq_state seq;
+    std::vector<uint16_t *> kp, vp;
+    char *ws = nullptr;
+    uint16_t *resid = nullptr, *q = nullptr, *attn = nullptr, *mlp = nullptr;
+    float2 *rope_cs = nullptr;
+    unsigned long long *best = nullptr;
+    unsigned *arrive = nullptr;
+    char *attn_ws = nullptr;
+    AttnWs attn_layout = {};
+    cudaStream_t cap = nullptr;
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    bool pdl = false;
+    int unpack = UNPACK_EXACT;
+    int n_kernels = 0;
+};
+
+static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1) {
+    const i4_model_desc &d = g->d;
+    const int H = d.hidden, I = d.intermediate, D = d.head_dim;
+    const int nqkv = (d.n_q_heads + 2 * d.n_kv_heads) * D;
+    const int max_pages = d.max_ctx / d.page_size;
+    int n = 0, st_ = 0;
+    auto pdl = [&]() { return g->pdl && n > 0 && only < 0; };
+    auto skip = [&]() { return only >= 0 && only != n; };
+    for (int l = 0; l < d.n_layers; ++l) {
+        const i4_layer_weights &L = g->layers[l];
+        {  // qkv + RoPE + KV append
+            GemvArgs a = {};
+            a.w = L.w_qkv;
+            a.s = L.s_qkv;
+            a.N = nqkv;
+            a.K = H;
+            a.M = 1;
+            a.x = l == 0 ? g->w.embed : g->resid;
+            a.gamma = L.ln_in;
+            a.eps = d.rms_eps;
+            a.token = g->seq.token;
+            a.vocab = d.vocab;
+            a.resid_out = g->resid;
+            a.bias = L.b_qkv;
+            a.pos = g->seq.pos;
+            a.page_table = g->seq.page_table;
+            a.k_pool = g->kp[l];
+            a.v_pool = g->vp[l];
+            a.q_out = g->q;
+            a.rope_cs = g->rope_cs;
+            a.n_q = d.n_q_heads;
+            a.n_kv = d.n_kv_heads;
+            a.page_size = d.page_size;
+            a.max_ctx = d.max_ctx;
+            a.status = g->seq.status;
+            if (!skip() && (st_ = launch_gemv(l == 0 ? PRO_EMBED : PRO_RMSNORM, EPI_ROPE_KV, a, st, pdl(), g->unpack, 0))) return st_;
+            ++n;
+        }
+        {  // attention
+            AttnParams p = {};
+            p.q = g->q;
+            p.k_pool = g->kp[l];
+            p.v_pool = g->vp[l];
+            p.page_table = g->seq.page_table;
+            p.ctx_len = g->seq.ctx_len;
+            p.out = g->attn;
+            p.B = 1;
+            p.Hq = d.n_q_heads;
+            p.Hkv = d.n_kv_heads;
+            p.page_size = d.page_size;
+            p.max_pages = max_pages;
+            p.splits = g->attn_layout.splits;
+            p.scale = (float)(1.0 / std::sqrt((double)D));
+            p.ws = g->attn_ws;
+            p.counters_off = g->attn_layout.counters_off;
+            p.ml_off = g->attn_layout.ml_off;
+            p.acc_off = g->attn_layout.acc_off;
+            if (!skip() && (st_ = launch_paged_gqa_decode(p, st, pdl()))) return st_;
+            ++n;
+        }
+        {  // o projection + residual
+            GemvArgs a = {};
+            a.w = L.w_o;
+            a.s = L.s_o;
+            a.N = H;
+            a.K = d.n_q_heads * D;
+            a.M = 1;
+            a.x = g->attn;
+            a.y = g->resid;
+            if (!skip() && (st_ = launch_gemv(PRO_PLAIN, EPI_RESID, a, st, pdl(), g->unpack, 0))) return st_;
+            ++n;
+        }
+        {  // RMSNorm + gate/up + SiLU-mul
+            GemvArgs a = {};
+            a.w = L.w_gate_up;
+            a.s = L.s_gate_up;
+            a.N = 2 * I;
+            a.K = H;
+            a.M = 1;
+            a.x = g->resid;
+            a.gamma = L.ln_post;
+            a.eps = d.rms_eps;
+            a.y = g->mlp;
+            a.inter = I;
+            if (!skip() && (st_ = launch_gemv(PRO_RMSNORM, EPI_SILU, a, st, pdl(), g->unpack, 0))) return st_;
+            ++n;
+        }
+        {  // down projection + residual
+            GemvArgs a = {};
+            a.w = L.w_down;
+            a.s = L.s_down;
+            a.N = H;
+            a.K = I;
+            a.M = 1;
+            a.x = g->mlp;
+            a.y = g->resid;
+            if (!skip() && (st_ = launch_gemv(PRO_PLAIN, EPI_RESID, a, st, pdl(), g->unpack, 0))) return st_;
+            ++n;
+        }
+    }
+    {  // final norm + lm_head + argmax + state advance
+        GemvArgs a = {};
+        a.w = g->w.w_lm;
+        a.s = g->w.s_lm;
+        a.N = d.vocab;
+        a.K = H;
+        a.M = 1;
+        a.x = g->resid;
+        a.gamma = g->w.ln_final;
+        a.eps = d.rms_eps;
+        a.y = g->seq.logits;
+        a.best = g->best;
+        a.arrive = g->arrive;
+        a.token_io = g->seq.token;
+        a.pos_io = g->seq.pos;
+        a.ctx_io = g->seq.ctx_len;
+        a.prompt = g->seq.prompt;
+        a.n_prompt = g->seq.prompt ? g->seq.n_prompt : 0;
+        a.history = g->seq.history;
+        a.max_ctx = d.max_ctx;
+        a.status = g->seq.status;
+        if (!skip() && (st_ = launch_gemv(PRO_RMSNORM, EPI_ARGMAX, a, st, pdl(), g->unpack, 0))) return st_;
+        ++n;
+    }
+    if (count) *count = n;
+    return I4_OK;
+}
+
+static int validate(const i4_model_desc *d, const i4_model_weights *w, const i4_seq_state *s) {
+    if (!d || !w || !s) return fail(I4_EINVAL, "decode_step_graph_create: null descriptor");
+    if (d->n_layers < 1 || d->hidden < 128 || d->intermediate < 128 || d->vocab < 1 || d->n_q_heads < 1 ||
+        d->n_kv_heads < 1 || d->max_ctx < 1 || d->page_size < 1)
+        return fail(I4_EINVAL, "model: non-positive size");
+    if (d->group != 128) return fail(I4_EUNSUPPORTED, "model: group %d (only 128)", d->group);
+    if (d->head_dim != 128) return fail(I4_EUNSUPPORTED, "model: head_dim %d (only 128)", d->head_dim);
+    if (d->hidden % 128 || d->intermediate % 128 || d->hidden > 32768 || d->intermediate > 32768)
+        return fail(I4_EUNSUPPORTED, "model: hidden and intermediate must be multiples of 128 up to 32768");
+    if (d->n_q_heads % d->n_kv_heads || d->n_q_heads / d->n_kv_heads > 8)
+        return fail(I4_EUNSUPPORTED, "model: n_q_heads / n_kv_heads must be an integer <= 8");
+    if ((d->n_q_heads * d->head_dim) % 128 || d->n_q_heads * d->head_dim > 32768)
+        return fail(I4_EUNSUPPORTED, "model: n_q_heads * head_dim");
+    if (d->page_size < 8 || d->page_size > 256 || (d->page_size & (d->page_size - 1)))
+        return fail(I4_EUNSUPPORTED, "model: page_size %d must be a power of two in [8, 256]", d->page_size);
+    if (d->max_ctx % d->page_size) return fail(I4_EINVAL, "model: max_ctx must be a multiple of page_size");
+    if (!(d->rms_eps >= 0.f) || !(d->rope_theta > 0.f)) return fail(I4_EINVAL, "model: eps/theta");
+    if (!w->embed || !w->layers || !w->ln_final || !w->w_lm || !w->s_lm) return fail(I4_EINVAL, "weights: null");
+    if (!aligned(w->embed, 16) || !aligned(w->ln_final, 16) || !aligned(w->w_lm, 16))
+        return fail(I4_EALIGN, "weights: 16-byte alignment");
+    for (int l = 0; l < d->n_layers; ++l) {
+        const i4_layer_weights &L = w->layers[l];
+        if (!L.w_qkv || !L.s_qkv || !L.b_qkv || !L.w_o || !L.s_o || !L.w_gate_up || !L.s_gate_up || !L.w_down ||
+            !L.s_down || !L.ln_in || !L.ln_post)
+            return fail(I4_EINVAL, "weights: null pointer in layer %d", l);
+        if (!aligned(L.w_qkv, 16) || !aligned(L.w_o, 16) || !aligned(L.w_gate_up, 16) || !aligned(L.w_down, 16) ||
+            !aligned(L.ln_in, 16) || !aligned(L.ln_post, 16))
+            return fail(I4_EALIGN, "weights: 16-byte alignment in layer %d", l);
+    }
+    if (!s->token || !s->pos || !s->ctx_len || !s->page_table || !s->k_pools || !s->v_pools || !s->logits ||
+        !s->status)
+        return fail(I4_EINVAL, "seq: null pointer");
+    if (s->num_pages < d->max_ctx / d->page_size) return fail(I4_EINVAL, "seq: pools hold fewer pages than max_ctx needs");
+    if (s->prompt && (s->n_prompt < 1 || s->n_prompt > d->max_ctx)) return fail(I4_EINVAL, "seq: n_prompt");
+    for (int l = 0; l < d->n_layers; ++l)
+        if (!s->k_pools[l] || !s->v_pools[l] || !aligned(s->k_pools[l], 16) || !aligned(s->v_pools[l], 16))
+            return fail(I4_EINVAL, "seq: pool of layer %d null or misaligned", l);
+    return I4_OK;
+}
+
+static void release(i4_graph *g) {
+    if (!g) return;
+    if (g->exec) cudaGraphExecDestroy(g->exec);
+    if (g->graph) cudaGraphDestroy(g->graph);
+    if (g->cap) cudaStreamDestroy(g->cap);
+    if (g->ws) cudaFree(g->ws);
+    delete g;
+}
+
+static size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+extern "C" int decode_step_graph_create(const i4_model_desc *desc, const i4_model_weights *weights,
+                                        const i4_seq_state *seq, i4_graph **out) {
+    if (!out) return fail(I4_EINVAL, "decode_step_graph_create: out is null");
+    *out = nullptr;
+    int st = validate(desc, weights, seq);
+    if (st) return st;
+    const int pages = desc->max_ctx / desc->page_size;
+    {  // every page id of the table must index the pools
+        std::vector<int32_t> tab(pages);
+        cudaError_t e = cudaMemcpy(tab.data(), seq->page_table, sizeof(int32_t) * pages, cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_check(e, "decode_step_graph_create: reading the page table");
+        for (int i = 0; i < pages; ++i)
+            if (tab[i] < 0 || tab[i] >= seq->num_pages)
+                return fail(I4_EINVAL, "seq: page_table[%d] = %d outside [0, %d)", i, tab[i], seq->num_pages);
+    }
+    i4_graph *g = new i4_graph();
+    g->d = *desc;
+    g->w = *weights;
+    g->layers.assign(weights->layers, weights->layers + desc->n_layers);
+    g->w.layers = g->layers.data();
+    g->seq = *seq;
+    g->kp.assign(seq->k_pools, seq->k_pools + desc->n_layers);
+    g->vp.assign(seq->v_pools, seq->v_pools + desc->n_layers);
+    g->seq.k_pools = g->kp.data();
+    g->seq.v_pools = g->vp.data();
+    g->pdl = g_pdl;
+    g->unpack = g_default_unpack;
+
+    const int H = desc->hidden, D = desc->head_dim;
+    g->attn_layout = attn_ws_layout(1, desc->n_q_heads, desc->n_kv_heads, desc->page_size, pages);
+    size_t off = 0;
+    const size_t o_resid = off; off += a256((size_t)H * 2);
+    const size_t o_q = off; off += a256((size_t)desc->n_q_heads * D * 2);
+    const size_t o_attn = off; off += a256((size_t)desc->n_q_heads * D * 2);
+    const size_t o_mlp = off; off += a256((size_t)desc->intermediate * 2);
+    const size_t o_rope = off; off += a256((size_t)desc->max_ctx * (D / 2) * sizeof(float2));
+    const size_t o_best = off; off += 256;
+    const size_t o_attn_ws = off; off += a256(g->attn_layout.bytes);
+    if (cudaMalloc(&g->ws, off) != cudaSuccess) {
+        cudaGetLastError();
+        release(g);
+        return fail(I4_ENOMEM, "decode_step_graph_create: cudaMalloc(%zu) failed", off);
+    }
+    g->resid = reinterpret_cast<uint16_t *>(g->ws + o_resid);
+    g->q = reinterpret_cast<uint16_t *>(g->ws + o_q);
+    g->attn = reinterpret_cast<uint16_t *>(g->ws + o_attn);
+    g->mlp = reinterpret_cast<uint16_t *>(g->ws + o_mlp);
+    g->rope_cs = reinterpret_cast<float2 *>(g->ws + o_rope);
+    g->best = reinterpret_cast<unsigned long long *>(g->ws + o_best);
+    g->arrive = reinterpret_cast<unsigned *>(g->ws + o_best + 8);
+    g->attn_ws = g->ws + o_attn_ws;
+
+    if ((st = cuda_check(cudaStreamCreateWithFlags(&g->cap, cudaStreamNonBlocking), "stream create")) ||
+        (st = cuda_check(cudaMemsetAsync(g->ws, 0, off, g->cap), "workspace clear")) ||
+        (st = launch_rope_table(g->rope_cs, desc->max_ctx, D, (double)desc->rope_theta, g->cap)) ||
+        (st = cuda_check(cudaStreamSynchronize(g->cap), "workspace init"))) {
+        release(g);
+        return st;
+    }
+    // configure every kernel variant (shared-memory limits, occupancy) outside the capture
+    g_dry_run = true;
+    st = enqueue_step(g, g->cap, &g->n_kernels);
+    g_dry_run = false;
+    if (st) {
+        release(g);
+        return st;
+    }
+    if ((st = cuda_check(cudaStreamBeginCapture(g->cap, cudaStreamCaptureModeThreadLocal), "begin capture"))) {
+        release(g);
+        return st;
+    }
+    st = enqueue_step(g, g->cap, nullptr);
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamEndCapture(g->cap, &graph);
+    g->graph = graph;
+    if (st || (st = cuda_check(e, "end capture")) ||
+        (st = cuda_check(cudaGraphInstantiate(&g->exec, g->graph, 0), "graph instantiate"))) {
+        release(g);
+        return st;
+    }
+    *out = g;
+    return I4_OK;
+}
+
+extern "C" int decode_step_graph_replay(i4_graph *g, void *stream) {
+    if (!g || !g->exec) return fail(I4_EINVAL, "decode_step_graph_replay: no graph");
+    return cuda_check(cudaGraphLaunch(g->exec, (cudaStream_t)stream), "graph launch");
+}
+
+extern "C" int decode_step_eager(i4_graph *g, void *stream) {
+    if (!g) return fail(I4_EINVAL, "decode_step_eager: no graph");
+    return enqueue_step(g, (cudaStream_t)stream, nullptr);
+}
+
+extern "C" int decode_step_kernel_count(const i4_graph *g) { return g ? g->n_kernels : 0; }
+
+extern "C" int decode_step_launch_kernel(i4_graph *g, int index, void *stream) {
+    if (!g) return fail(I4_EINVAL, "decode_step_launch_kernel: no graph");
+    if (index < 0 || index >= g->n_kernels)
+        return fail(I4_EINVAL, "decode_step_launch_kernel: index %d outside [0, %d)", index, g->n_kernels);
+    return enqueue_step(g, (cudaStream_t)stream, nullptr, index);
+}
+
+extern "C" int decode_step_graph_destroy(i4_graph *g) {
+    if (!g) return fail(I4_EINVAL, "decode_step_graph_destroy: null");
+    release(g);
+    return I4_OK;
+}
+
+// Library options: "pdl" (programmatic dependent launch inside the decode step,
+// 0/1) and "unpack" (GEMV unpack variant, 0 exact / 1 subnormal). They apply to
+// graphs created afterwards and to int4_gemv calls.
+extern "C" int i4_set_option(const char *name, int value) {
+    if (!name) return fail(I4_EINVAL, "i4_set_option: null name");
+    const std::string n(name);
+    if (n == "pdl") {
+        g_pdl = value != 0;
+        return I4_OK;
+    }
+    if (n == "unpack") {
+        if (value != UNPACK_EXACT && value != UNPACK_SUBNORMAL) return fail(I4_EINVAL, "unpack must be 0 or 1");
+        g_default_unpack = value;
+        return I4_OK;
+    }
+    return fail(I4_EINVAL, "i4_set_option: unknown option '%s'", name);
+}

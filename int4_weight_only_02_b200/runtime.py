@@ -1,0 +1,151 @@
+"""Device-side model, sequence state and the captured decode step (argument marshalling only).
+
+``DeviceModel`` holds the INT4 weights of a Qwen2.5-7B-shaped decoder in HBM,
+``Sequence`` one sequence's paged KV pools and on-device decode state, and
+``DecodeGraph`` the decode step of ``libi4rt`` (one CUDA graph per token,
+``decode_step_graph_*``). PyTorch only allocates the memory.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import (LayerWeights, ModelDesc, ModelWeights, SeqState, _check, _p, _stream, lib, synth)
+
+_LAYER_KEYS = ("w_qkv", "s_qkv", "b_qkv", "w_o", "s_o", "w_gu", "s_gu", "w_d", "s_d", "ln_in", "ln_post")
+_LAYER_FIELDS = ("w_qkv", "s_qkv", "b_qkv", "w_o", "s_o", "w_gate_up", "s_gate_up", "w_down", "s_down", "ln_in",
+                 "ln_post")
+
+
+def to_device(a: np.ndarray, device="cuda"):
+    """Upload a numpy array; uint32 words travel as int32 (same bits)."""
+    import torch
+    if a.dtype == np.uint32:
+        a = a.view(np.int32)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+class DeviceModel:
+    def __init__(self, shape: synth.ModelShape, layers, glob, device="cuda"):
+        self.shape = shape
+        self.device = device
+        self.layers = [{k: to_device(v, device) for k, v in lw.items()} for lw in layers]
+        self.glob = {k: to_device(v, device) for k, v in glob.items()}
+
+    @classmethod
+    def synthetic(cls, shape: synth.ModelShape = synth.QWEN7B, seed: int = 0, device="cuda"):
+        """Random-init weights of the given shape, generated and uploaded one layer at a time."""
+        self = cls.__new__(cls)
+        self.shape, self.device = shape, device
+        self.layers = []
+        for i in range(shape.layers):
+            self.layers.append({k: to_device(v, device) for k, v in synth.layer_weights(shape, i, seed).items()})
+        self.glob = {k: to_device(v, device) for k, v in synth.global_weights(shape, seed).items()}
+        return self
+
+    def weight_bytes(self) -> int:
+        """INT4 words + fp16 scales streamed per token (28 layers and lm_head)."""
+        n = 0
+        for lw in self.layers:
+            for k in ("w_qkv", "s_qkv", "w_o", "s_o", "w_gu", "s_gu", "w_d", "s_d"):
+                n += lw[k].numel() * lw[k].element_size()
+        for k in ("w_lm", "s_lm"):
+            n += self.glob[k].numel() * self.glob[k].element_size()
+        return n
+
+    def desc(self) -> ModelDesc:
+        s = self.shape
+        return ModelDesc(s.layers, s.hidden, s.inter, s.n_q, s.n_kv, s.head_dim, s.vocab, s.group, s.page_size,
+                         s.max_ctx, s.theta, s.eps)
+
+
+class Sequence:
+    """One sequence: K/V pools per layer, a page table, and the on-device decode state."""
+
+    def __init__(self, model: DeviceModel, page_table: np.ndarray, prompt: np.ndarray | None = None,
+                 num_pages: int | None = None):
+        import torch
+        s, dev = model.shape, model.device
+        self.model = model
+        self.num_pages = int(num_pages if num_pages is not None else s.max_pages)
+        kv = (self.num_pages, s.n_kv, s.page_size, s.head_dim)
+        self.k_pools = [torch.zeros(kv, dtype=torch.float16, device=dev) for _ in range(s.layers)]
+        self.v_pools = [torch.zeros(kv, dtype=torch.float16, device=dev) for _ in range(s.layers)]
+        self.page_table = to_device(np.asarray(page_table, dtype=np.int32), dev)
+        self.token = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.pos = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.ctx_len = torch.ones(1, dtype=torch.int32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.logits = torch.zeros(s.vocab, dtype=torch.float32, device=dev)
+        self.history = torch.zeros(s.max_ctx, dtype=torch.int32, device=dev)
+        self.prompt = None
+        if prompt is not None:
+            self.prompt = to_device(np.asarray(prompt, dtype=np.int32), dev)
+        self.reset()
+
+    def reset(self, first_token: int | None = None):
+        """Position 0 with the first prompt token (or `first_token`)."""
+        tok = first_token
+        if tok is None:
+            tok = int(self.prompt[0].item()) if self.prompt is not None else 0
+        self.token.fill_(tok)
+        self.pos.zero_()
+        self.ctx_len.fill_(1)
+        self.status.zero_()
+        self.history.zero_()
+        self.history[0] = tok
+
+    def state(self) -> SeqState:
+        self._kp = (ctypes.c_void_p * len(self.k_pools))(*[t.data_ptr() for t in self.k_pools])
+        self._vp = (ctypes.c_void_p * len(self.v_pools))(*[t.data_ptr() for t in self.v_pools])
+        return SeqState(self.token.data_ptr(), self.pos.data_ptr(), self.ctx_len.data_ptr(),
+                        self.page_table.data_ptr(), self._kp, self._vp, self.num_pages, self.logits.data_ptr(),
+                        self.prompt.data_ptr() if self.prompt is not None else None,
+                        int(self.prompt.numel()) if self.prompt is not None else 0,
+                        self.history.data_ptr(), self.status.data_ptr())
+
+
+class DecodeGraph:
+    """The decode step of libi4rt: ``replay()`` runs one token as one cudaGraphLaunch."""
+
+    def __init__(self, model: DeviceModel, seq: Sequence):
+        self.model, self.seq = model, seq
+        layers = (LayerWeights * len(model.layers))()
+        for i, lw in enumerate(model.layers):
+            for key, field in zip(_LAYER_KEYS, _LAYER_FIELDS):
+                setattr(layers[i], field, lw[key].data_ptr())
+        g = model.glob
+        weights = ModelWeights(g["embed"].data_ptr(), layers, g["ln_final"].data_ptr(), g["w_lm"].data_ptr(),
+                               g["s_lm"].data_ptr())
+        desc = model.desc()
+        state = seq.state()
+        handle = ctypes.c_void_p()
+        _check(lib().decode_step_graph_create(ctypes.byref(desc), ctypes.byref(weights), ctypes.byref(state),
+                                              ctypes.byref(handle)), "decode_step_graph_create")
+        self._h = handle
+
+    @property
+    def kernel_count(self) -> int:
+        return int(lib().decode_step_kernel_count(self._h))
+
+    def replay(self, stream=None):
+        _check(lib().decode_step_graph_replay(self._h, _stream(stream)), "decode_step_graph_replay")
+
+    def eager(self, stream=None):
+        _check(lib().decode_step_eager(self._h, _stream(stream)), "decode_step_eager")
+
+    def launch_kernel(self, index: int, stream=None):
+        """Launch only kernel `index` of the step (benchmarking; see decode_step_launch_kernel)."""
+        _check(lib().decode_step_launch_kernel(self._h, index, _stream(stream)), "decode_step_launch_kernel")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _check(lib().decode_step_graph_destroy(self._h), "decode_step_graph_destroy")
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -13,7 +13,12 @@ description of the 7B-shape decode benchmark):
 
 * packed INT4 weights: uniformly random uint32 words. Eight signed 4-bit
   fields per word, so every field is uniform over [-8, 7];
-* group scales: uniform in [0.005, 0.02], drawn in float64, rounded to fp16;
+* group scales: uniform in [0.005, 0.02], drawn in float64, rounded to fp16.
+  In the full decoder every group scale also gets a random sign: the codes
+  uniform over [-8, 7] have mean -1/2, so all-positive scales give every weight
+  matrix a common negative mean; through the MLP that mean feeds back from
+  layer to layer and the fp16 residual overflows to inf in the second layer.
+  Random signs make the mean zero and keep the 28-layer residual near 400 RMS;
 * activations, K/V, queries, embedding rows: N(0, 1), rounded to fp16;
 * qkv bias: N(0, 0.1), rounded to fp16;
 * RMSNorm weights (gamma): N(1, 0.1), rounded to fp16;
@@ -70,10 +75,13 @@ def packed_int4(rng: np.random.Generator, n: int, k: int) -> np.ndarray:
     return rng.integers(0, 2**32, size=(n, k // 8), dtype=np.uint32)
 
 
-def group_scales(rng: np.random.Generator, n: int, k: int, group: int = 128) -> np.ndarray:
-    """[n][k/group] fp16, uniform in [0.005, 0.02]."""
+def group_scales(rng: np.random.Generator, n: int, k: int, group: int = 128, signed: bool = False) -> np.ndarray:
+    """[n][k/group] fp16 with magnitudes uniform in [0.005, 0.02]; a random sign per group when `signed`."""
     assert k % group == 0
-    return rng.uniform(0.005, 0.02, size=(n, k // group)).astype(np.float16)
+    mag = rng.uniform(0.005, 0.02, size=(n, k // group))
+    if signed:
+        mag = mag * (2.0 * rng.integers(0, 2, size=mag.shape) - 1.0)
+    return mag.astype(np.float16)
 
 
 def normal_f16(rng: np.random.Generator, shape, mean: float = 0.0, std: float = 1.0) -> np.ndarray:
@@ -138,14 +146,14 @@ def layer_weights(shape: ModelShape, layer: int, seed: int = 0) -> dict:
     r = lambda code: rng_for(seed, layer, code)
     return {
         "w_qkv": packed_int4(r(W_QKV), nqkv, h),
-        "s_qkv": group_scales(r(S_QKV), nqkv, h, g),
+        "s_qkv": group_scales(r(S_QKV), nqkv, h, g, signed=True),
         "b_qkv": normal_f16(r(B_QKV), (nqkv,), 0.0, 0.1),
         "w_o": packed_int4(r(W_O), h, shape.n_q * shape.head_dim),
-        "s_o": group_scales(r(S_O), h, shape.n_q * shape.head_dim, g),
+        "s_o": group_scales(r(S_O), h, shape.n_q * shape.head_dim, g, signed=True),
         "w_gu": packed_int4(r(W_GU), 2 * i, h),
-        "s_gu": group_scales(r(S_GU), 2 * i, h, g),
+        "s_gu": group_scales(r(S_GU), 2 * i, h, g, signed=True),
         "w_d": packed_int4(r(W_D), h, i),
-        "s_d": group_scales(r(S_D), h, i, g),
+        "s_d": group_scales(r(S_D), h, i, g, signed=True),
         "ln_in": normal_f16(r(LN_IN), (h,), 1.0, 0.1),
         "ln_post": normal_f16(r(LN_POST), (h,), 1.0, 0.1),
     }
@@ -157,7 +165,7 @@ def global_weights(shape: ModelShape, seed: int = 0) -> dict:
         "embed": normal_f16(r(EMBED), (shape.vocab, shape.hidden)),
         "ln_final": normal_f16(r(LN_FINAL), (shape.hidden,), 1.0, 0.1),
         "w_lm": packed_int4(r(W_LM), shape.vocab, shape.hidden),
-        "s_lm": group_scales(r(S_LM), shape.vocab, shape.hidden, shape.group),
+        "s_lm": group_scales(r(S_LM), shape.vocab, shape.hidden, shape.group, signed=True),
     }
 
 

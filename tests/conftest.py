@@ -17,3 +17,22 @@ def pytest_configure(config):
 def oracle_lib():
     import oracle
     return oracle.lib()
+
+
+@pytest.fixture(scope="session")
+def i4lib():
+    """The built CUDA library (built in-tree on first use when missing or stale)."""
+    from int4_weight_only_02_b200 import build as b
+    b.build()
+    import int4_weight_only_02_b200 as i4
+    return i4
+
+
+@pytest.fixture(scope="session")
+def cuda(i4lib):
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for -m gpu tests")
+    torch.cuda.init()
+    return torch.device("cuda:0")
+

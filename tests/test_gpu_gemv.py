@@ -1,0 +1,106 @@
+"""INT4 GEMV and unpack through the C ABI vs the CPU oracle (needs a B200).
+
+Tolerance: the workload names a max relative error of 2e-3 for fp16 outputs
+with fp32 accumulation, read here as normwise max|g - r| / max|r| (the oracle
+sums in fp64). Both unpack variants are checked. Exact-arithmetic inputs
+(power-of-two scales, small integer x) must come out bit-exact.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from int4_weight_only_02_b200 import synth
+from helpers import dev, normwise_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+def run_gemv(i4, cuda, w, s, x, b=None, out_fp32=False, unpack=None):
+    y = i4.int4_gemv(dev(w, cuda), dev(s, cuda), dev(np.atleast_2d(x), cuda),
+                     None if b is None else dev(b, cuda), out_fp32=out_fp32, unpack=unpack)
+    import torch
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+def pack_fields(q):
+    n, k = q.shape
+    u = (q.astype(np.int64) & 0xF).reshape(n, k // 8, 8)
+    words = np.zeros((n, k // 8), dtype=np.int64)
+    for i in range(8):
+        words |= u[:, :, i] << (4 * i)
+    return words.astype(np.uint32)
+
+
+def test_unpack_bit_exact(i4lib, cuda):
+    rng = np.random.default_rng(0)
+    w = rng.integers(0, 2**32, size=(37, 64), dtype=np.uint32)
+    w[0, :16] = np.arange(16, dtype=np.uint32) * 0x11111111  # every code in every field
+    got = i4lib.int4_unpack(dev(w, cuda), 512).cpu().numpy()
+    assert np.array_equal(got, oracle.unpack_int4(w, 512))
+
+
+@pytest.mark.parametrize("unpack", [0, 1])
+def test_qkv_shape_against_oracle(i4lib, cuda, unpack):
+    w, s, x, b = synth.gemv_case(4608, 3584, seed=0, bias=True)
+    ref = oracle.int4_gemv(w, s, x[0], b)
+    got = run_gemv(i4lib, cuda, w, s, x, b, unpack=unpack)[0]
+    assert normwise_err(got, ref) <= TOL
+    assert np.mean(got == ref) >= 0.98  # fp32 vs fp64 sums round to the same fp16 almost always
+
+
+@pytest.mark.parametrize("unpack", [0, 1])
+def test_exact_arithmetic_is_bit_exact(i4lib, cuda, unpack):
+    rng = np.random.default_rng(1)
+    n, k = 96, 1024
+    q = rng.integers(-8, 8, size=(n, k))
+    s = np.ldexp(1.0, rng.integers(-8, -4, size=(n, k // 128))).astype(np.float16)
+    x = rng.integers(-3, 4, size=(1, k)).astype(np.float16)
+    w = pack_fields(q)
+    ref = oracle.int4_gemv(w, s, x[0], None)
+    got = run_gemv(i4lib, cuda, w, s, x, unpack=unpack)[0]
+    assert np.array_equal(got.view(np.uint16), ref.view(np.uint16))
+    got32 = run_gemv(i4lib, cuda, w, s, x, out_fp32=True, unpack=unpack)[0]
+    assert np.array_equal(got32, oracle.int4_linear(w, s, x[0]).astype(np.float32))
+
+
+@pytest.mark.parametrize("n,k,m", [(1, 128, 1), (37, 640, 1), (129, 384, 2), (64, 3584, 3), (50, 1152, 5),
+                                   (33, 256, 8)])
+def test_ragged_shapes_and_batches(i4lib, cuda, n, k, m):
+    w, s, x, b = synth.gemv_case(n, k, m=m, seed=3, bias=True)
+    ref = oracle.int4_gemv(w, s, x, b)
+    for unpack in (0, 1):
+        got = run_gemv(i4lib, cuda, w, s, x, b, unpack=unpack)
+        assert got.shape == (m, n)
+        assert normwise_err(got, ref) <= TOL
+
+
+def test_mlp_shapes_against_oracle(i4lib, cuda):
+    # gate/up K=3584 N=37888 and down K=18944 N=3584 (the MLP block of the 7B shape)
+    for n, k in [(37888, 3584), (3584, 18944)]:
+        w, s, x, _ = synth.gemv_case(n, k, seed=5)
+        ref = oracle.int4_gemv(w, s, x[0])
+        got = run_gemv(i4lib, cuda, w, s, x)[0]
+        assert normwise_err(got, ref) <= TOL, (n, k)
+
+
+def test_lm_head_fp32_logits(i4lib, cuda):
+    w, s, x, _ = synth.gemv_case(152064, 3584, seed=6)
+    ref = oracle.int4_linear(w, s, x[0])
+    got = run_gemv(i4lib, cuda, w, s, x, out_fp32=True)[0]
+    assert got.dtype == np.float32
+    assert normwise_err(got, ref) <= 1e-5
+    assert int(np.argmax(got)) == oracle.argmax(ref.astype(np.float32))
+
+
+def test_bad_arguments_raise(i4lib, cuda):
+    import torch
+    w, s, x, _ = synth.gemv_case(8, 256, seed=7)
+    wd, sd = dev(w, cuda), dev(s, cuda)
+    xd = dev(x, cuda)
+    with pytest.raises(i4lib.I4Error):
+        i4lib.int4_gemv(wd, sd, xd, group=64)
+    with pytest.raises(i4lib.I4Error):
+        i4lib.int4_gemv(wd, sd, torch.zeros((9, 256), dtype=torch.float16, device=cuda))
