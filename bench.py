@@ -318,6 +318,8 @@ def main():
     def time_kernel(index_fn, reps=2):
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(shape.layers * reps)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(shape.layers * reps)]
+        torch.cuda.synchronize()
+        torch.cuda._sleep(100_000_000)  # keep the GPU busy while the host queues every launch
         for r in range(reps):
             for li in range(shape.layers):
                 j = r * shape.layers + li

@@ -93,7 +93,7 @@ I4_API int i4_int4_unpack(const uint32_t *w, int8_t *q, int N, int K, void *stre
  *               leaves its counters zero again. Calls sharing one ws must not
  *               overlap on the GPU.
  * Requires D == 128, 1 <= Hq / Hkv <= 8 (Hq % Hkv == 0), page_size a power of
- * two in [8, 256], B >= 1.
+ * two in [8, 128], max_pages_per_seq * page_size <= 32768, B >= 1.
  */
 I4_API size_t paged_gqa_decode_ws_bytes(int B, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq);
 I4_API int paged_gqa_decode(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_pool, const int32_t *page_table,
@@ -241,14 +241,25 @@ I4_API int decode_step_launch_kernel(i4_graph *g, int index, void *stream);
  *            dependent launch (each kernel still waits for its predecessor's
  *            results before reading them);
  *   "unpack" 0/1: INT4 unpack variant of the GEMV (0 exact fp16 values,
- *            1 offset-binary fp16 subnormals with a per-chunk sum(x) correction).
+ *            1 offset-binary fp16 subnormals with a per-chunk sum(x) correction);
+ *   "stream" 0/1: use the bulk-copy pipelined GEMV where the shape allows it
+ *            (M == 1, K % 512 == 0, 16-byte aligned w and scales), default 1;
+ *   "stream_smem_kb" 32..227: shared memory budget of that kernel's ring.
  * Not thread-safe; set options before creating graphs.
  */
 I4_API int i4_set_option(const char *name, int value);
 
 /*
+ * Device-side error flag: 0, or 1 when a bounded wait inside a kernel gave up
+ * (the kernel then stopped early and its outputs are invalid). Synchronises
+ * with the device; reset != 0 clears the flag. Negative on a CUDA error.
+ */
+I4_API int i4_device_error(int reset);
+
+/*
  * int4_gemv with an explicit unpack variant (0 or 1, as above) and a cap on the
- * number of CTAs (0 = none); for tests and benchmarks.
+ * number of CTAs (0 = none; any cap selects the register-streaming kernel
+ * instead of the bulk-copy pipelined one); for tests and benchmarks.
  */
 I4_API int i4_int4_gemv_variant(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
                          int y_is_fp32, int M, int N, int K, int unpack, int max_ctas, void *stream);

@@ -81,6 +81,7 @@ _SIGS = {
     "decode_step_graph_destroy": (_i, [_vp]),
     "decode_step_launch_kernel": (_i, [_vp, _i, _vp]),
     "i4_set_option": (_i, [ctypes.c_char_p, _i]),
+    "i4_device_error": (_i, [_i]),
 }
 
 
@@ -117,6 +118,14 @@ def _stream(stream):
     import torch
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def device_error(reset: bool = True) -> int:
+    """0, or 1 when a bounded in-kernel wait gave up (synchronises the device)."""
+    v = int(lib().i4_device_error(int(reset)))
+    if v < 0:
+        _check(v, "i4_device_error")
+    return v
 
 
 def set_option(name: str, value: int):

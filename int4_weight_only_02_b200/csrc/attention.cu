@@ -5,21 +5,28 @@
 // paged KV cache and attention; lessons: a __syncthreads() inside a
 // warp-specialised branch corrupted the softmax at KV-page tails). The H100
 // design there was warp-specialised with TMA; at batch 1 a decode head reads
-// well under 1 MB, so this kernel has no producer/consumer roles at all: every
-// thread of a CTA runs the same three phases, and every barrier is reached by
-// the whole CTA (CTAs without work leave before the first barrier, as a whole).
+// well under 1 MB, so this kernel has no producer/consumer roles: thread 0
+// issues one bulk copy (cp.async.bulk, no multicast) per K page and per V page
+// of the CTA's range into shared memory, every thread then runs the same
+// three phases, and every barrier is reached by the whole CTA (CTAs without
+// work leave before the first barrier, as a whole).
 //
 // Grid (S, Hkv, B). CTA (s, g, b) takes pages [s*pps, (s+1)*pps) of sequence b
 // for kv head g and all G = Hq/Hkv query heads that share it, so each K/V row
 // is read once for G heads. pps is derived on the device from ctx_len[b], so a
-// captured graph stays valid as the context grows.
-//   phase A: 16 threads per token (8 dims each, one 16-byte load of K),
-//            8 tokens per pass; scores = q.k * scale * log2(e) into shared memory.
+// captured graph stays valid as the context grows. One page of one kv head is
+// page_size contiguous rows of 256 bytes, so a page is one copy.
+//   phase A: 16 threads per token (8 dims each), 8 tokens per pass;
+//            scores = q.k * scale * log2(e) into shared memory.
 //   phase B: per head, max and sum of exp2 over the CTA's tokens.
 //   phase C: o[h][:] += p[h][t] * V[t][:], same thread layout as phase A.
 // With one active split the CTA writes the normalised output; otherwise it
 // writes (m, l, o) partials and the last CTA to arrive for (b, g) merges them:
 //   M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+// Pages below the current token's page were written by earlier decode steps,
+// so their copies start before the dependency wait (programmatic launch); the
+// page holding position ctx-1 is copied after it.
+#include "async.cuh"
 #include "attention.cuh"
 #include "common.cuh"
 
@@ -28,11 +35,13 @@ namespace i4 {
 constexpr int kAttnThreads = 128;
 constexpr int kMaxGroup = 8;
 constexpr int kHeadDim = 128;
-constexpr int kMaxTokensPerSplit = 512;
+constexpr int kMaxTokensPerSplit = 128;
 constexpr int kMinTokensPerSplit = 32;
-constexpr int kMaxSplits = kMaxTokensPerSplit;  // the merge keeps one weight per split in the score buffer
+constexpr int kMaxSplits = 256;
 constexpr int kMaxCtx = kMaxSplits * kMaxTokensPerSplit;
 constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ int g_attn_error = 0;
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -59,13 +68,21 @@ AttnWs attn_ws_layout(int B, int Hq, int Hkv, int page_size, int max_pages) {
     return L;
 }
 
+// Largest token range one CTA can be given: the shared-memory K and V tiles are this long.
+static int attn_tile_tokens(const AttnParams &p) {
+    const int min_pps = (kMinTokensPerSplit + p.page_size - 1) / p.page_size;
+    int pps = (p.max_pages + p.splits - 1) / p.splits;
+    pps = pps < min_pps ? min_pps : pps;
+    return pps * p.page_size;
+}
+
 __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnParams p) {
-    grid_dep_wait();
+    extern __shared__ __align__(128) unsigned char kv_smem[];
     const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int G = p.Hq / p.Hkv;
     const int P = p.page_size;
     const int max_ctx = p.max_pages * P;
-    int ctx = p.ctx_len[b];
+    int ctx = p.ctx_len[b];  // written by an earlier step, never by this kernel's predecessor
     ctx = ctx < 1 ? 1 : (ctx > max_ctx ? max_ctx : ctx);
     const int n_pages = (ctx + P - 1) / P;
     const int min_pps = (kMinTokensPerSplit + P - 1) / P;
@@ -77,15 +94,47 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
     __shared__ float qs[kMaxGroup][kHeadDim];
     __shared__ float sc[kMaxGroup][kMaxTokensPerSplit];
     __shared__ float red[4][kMaxGroup][kHeadDim];
+    __shared__ float coef[kMaxGroup][kMaxSplits];
     __shared__ float mh[kMaxGroup], lh[kMaxGroup];
+    __shared__ __align__(8) uint64_t kbar, vbar;
     __shared__ int is_last;
 
     const int tid = threadIdx.x;
-    const int t0 = s * pps * P;
-    const int t1 = (t0 + pps * P) < ctx ? (t0 + pps * P) : ctx;
+    const int p0 = s * pps;
+    const int p1 = (p0 + pps) < n_pages ? (p0 + pps) : n_pages;
+    const int t0 = p0 * P;
+    const int t1 = (p1 * P) < ctx ? (p1 * P) : ctx;
     const int T = t1 - t0;
     const int32_t *table = p.page_table + (size_t)b * p.max_pages;
     const float qscale = p.scale * kLog2e;
+    const unsigned page_bytes = (unsigned)P * kHeadDim * 2;
+    unsigned char *ks = kv_smem;                                   // [tile tokens][128] fp16
+    unsigned char *vs = kv_smem + (size_t)p.tile_tokens * kHeadDim * 2;
+    const int last_page = n_pages - 1;                            // holds position ctx-1
+
+    if (tid == 0) {
+        mbar_init(&kbar, 1);
+        mbar_init(&vbar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const uint64_t pol = evict_first_policy();
+    if (tid == 0) {
+        mbar_expect_tx(&kbar, (unsigned)(p1 - p0) * page_bytes);
+        mbar_expect_tx(&vbar, (unsigned)(p1 - p0) * page_bytes);
+        for (int pg = p0; pg < p1; ++pg) {
+            if (pg == last_page) continue;
+            const size_t off = ((size_t)table[pg] * p.Hkv + g) * P * kHeadDim;
+            bulk_load(ks + (size_t)(pg - p0) * page_bytes, p.k_pool + off, page_bytes, &kbar, pol);
+            bulk_load(vs + (size_t)(pg - p0) * page_bytes, p.v_pool + off, page_bytes, &vbar, pol);
+        }
+    }
+    grid_dep_wait();  // q and the current token's K/V row come from the preceding kernel
+    if (tid == 0 && last_page >= p0 && last_page < p1) {
+        const size_t off = ((size_t)table[last_page] * p.Hkv + g) * P * kHeadDim;
+        bulk_load(ks + (size_t)(last_page - p0) * page_bytes, p.k_pool + off, page_bytes, &kbar, pol);
+        bulk_load(vs + (size_t)(last_page - p0) * page_bytes, p.v_pool + off, page_bytes, &vbar, pol);
+    }
 
     // q of the G heads, fp32, pre-scaled
     for (int i = tid; i < G * kHeadDim; i += kAttnThreads) {
@@ -93,6 +142,8 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
         qs[h][d] = half_bits_to_float(p.q[((size_t)b * p.Hq + g * G + h) * kHeadDim + d]) * qscale;
     }
     __syncthreads();
+    bool ok = mbar_wait(&kbar, 0);
+    if (!ok) record_error(&g_attn_error, 1);
 
     const int tk = tid >> 4;         // token lane 0..7
     const int dl = tid & 15;         // 8 dims [8dl, 8dl+8)
@@ -104,14 +155,11 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
 #pragma unroll
             for (int e = 0; e < 8; ++e) qr[h][e] = h < G ? qs[h][8 * dl + e] : 0.f;
         // every lane runs the same passes (the shuffles below need the full warp)
-        for (int tb = t0; tb < t1; tb += 8) {
+        for (int tb = 0; tb < T; tb += 8) {
             const int t = tb + tk;
-            const bool live = t < t1;
+            const bool live = t < T;
             uint4 kv = make_uint4(0, 0, 0, 0);
-            if (live) {
-                const size_t row = ((size_t)table[t / P] * p.Hkv + g) * P + (t % P);
-                kv = *reinterpret_cast<const uint4 *>(p.k_pool + row * kHeadDim + 8 * dl);
-            }
+            if (live && ok) kv = *reinterpret_cast<const uint4 *>(ks + ((size_t)t * kHeadDim + 8 * dl) * 2);
             const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
             float kf[8];
 #pragma unroll
@@ -127,7 +175,7 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
                 for (int e = 0; e < 8; ++e) d = fmaf(qr[h][e], kf[e], d);
 #pragma unroll
                 for (int o = 8; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-                if (live && dl == 0 && h < G) sc[h][t - t0] = d;
+                if (live && dl == 0 && h < G) sc[h][t] = d;
             }
         }
     }
@@ -155,6 +203,10 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
         }
     }
     __syncthreads();
+    if (!mbar_wait(&vbar, 0)) {
+        record_error(&g_attn_error, 1);
+        ok = false;
+    }
 
     // ---- phase C: o = sum_t p_t v_t
     float acc[kMaxGroup][8];
@@ -162,9 +214,8 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
     for (int h = 0; h < kMaxGroup; ++h)
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
-    for (int t = t0 + tk; t < t1; t += 8) {
-        const size_t row = ((size_t)table[t / P] * p.Hkv + g) * P + (t % P);
-        const uint4 vv = *reinterpret_cast<const uint4 *>(p.v_pool + row * kHeadDim + 8 * dl);
+    for (int t = tk; t < T && ok; t += 8) {
+        const uint4 vv = *reinterpret_cast<const uint4 *>(vs + ((size_t)t * kHeadDim + 8 * dl) * 2);
         const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
         float vf[8];
 #pragma unroll
@@ -176,7 +227,7 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
 #pragma unroll
         for (int h = 0; h < kMaxGroup; ++h) {
             if (h < G) {
-                const float pt = sc[h][t - t0];
+                const float pt = sc[h][t];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(pt, vf[e], acc[h][e]);
             }
@@ -227,8 +278,6 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
     if (!is_last) return;
     __threadfence();
 
-    // per-split weight / L, in the score buffer (no longer read by anyone); splits <= kMaxSplits
-    float (*coef)[kMaxTokensPerSplit] = sc;
     if (tid < G) {
         const int h = tid;
         float M = -INFINITY;
@@ -254,11 +303,32 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
     if (tid == 0) *counter = 0u;  // ready for the next call
 }
 
-int launch_paged_gqa_decode(const AttnParams &p, cudaStream_t stream, bool pdl) {
+int launch_paged_gqa_decode(const AttnParams &p_in, cudaStream_t stream, bool pdl) {
+    AttnParams p = p_in;
+    p.tile_tokens = attn_tile_tokens(p);
+    const int smem = 2 * p.tile_tokens * kHeadDim * 2;
+    static int configured = -1;
+    if (smem > configured) {
+        cudaError_t e = cudaFuncSetAttribute(paged_gqa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_check(e, "paged_gqa_decode smem attribute");
+        configured = smem;
+    }
     if (g_dry_run) return I4_OK;
-    return cuda_check(launch(paged_gqa_decode_kernel, dim3(p.splits, p.Hkv, p.B), dim3(kAttnThreads), 0, stream,
-                             pdl, p),
+    return cuda_check(launch(paged_gqa_decode_kernel, dim3(p.splits, p.Hkv, p.B), dim3(kAttnThreads), (size_t)smem,
+                             stream, pdl, p),
                       "paged_gqa_decode launch");
+}
+
+int read_attn_error(int reset) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_attn_error, sizeof v);
+    if (e != cudaSuccess) return cuda_check(e, "reading the attention error flag");
+    if (reset && v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_attn_error, &zero, sizeof zero);
+        if (e != cudaSuccess) return cuda_check(e, "clearing the attention error flag");
+    }
+    return v;
 }
 
 // out[b][g][t][:] = pool row of token t, t < ctx_len[b]
@@ -289,8 +359,9 @@ static int attn_check(const uint16_t *q, const uint16_t *k_pool, const uint16_t 
     if (B < 1 || Hq < 1 || Hkv < 1 || max_pages < 1) return fail(I4_EINVAL, "paged_gqa_decode: bad sizes");
     if (D != 128) return fail(I4_EUNSUPPORTED, "paged_gqa_decode: head_dim %d (only 128)", D);
     if (Hq % Hkv != 0 || Hq / Hkv > 8) return fail(I4_EUNSUPPORTED, "paged_gqa_decode: Hq/Hkv must be an integer <= 8");
-    if (page_size < 8 || page_size > 256 || (page_size & (page_size - 1)))
-        return fail(I4_EUNSUPPORTED, "paged_gqa_decode: page_size %d must be a power of two in [8, 256]", page_size);
+    if (page_size < 8 || page_size > kMaxTokensPerSplit || (page_size & (page_size - 1)))
+        return fail(I4_EUNSUPPORTED, "paged_gqa_decode: page_size %d must be a power of two in [8, %d]", page_size,
+                    kMaxTokensPerSplit);
     if (B > 65535 || Hkv > 65535) return fail(I4_EUNSUPPORTED, "paged_gqa_decode: grid too large");
     if ((long long)max_pages * page_size > kMaxCtx)
         return fail(I4_EUNSUPPORTED, "paged_gqa_decode: max_pages_per_seq * page_size above %d tokens", kMaxCtx);

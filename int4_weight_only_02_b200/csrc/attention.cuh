@@ -10,6 +10,7 @@ struct AttnParams {
     const int32_t *page_table, *ctx_len;
     uint16_t *out;
     int B, Hq, Hkv, page_size, max_pages, splits;
+    int tile_tokens;  // K/V shared-memory tile length (set by the launcher)
     float scale;
     char *ws;
     size_t counters_off, ml_off, acc_off;

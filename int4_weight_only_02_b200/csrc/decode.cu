@@ -195,8 +195,9 @@ static int validate(const i4_model_desc *d, const i4_model_weights *w, const i4_
         return fail(I4_EUNSUPPORTED, "model: n_q_heads / n_kv_heads must be an integer <= 8");
     if ((d->n_q_heads * d->head_dim) % 128 || d->n_q_heads * d->head_dim > 32768)
         return fail(I4_EUNSUPPORTED, "model: n_q_heads * head_dim");
-    if (d->page_size < 8 || d->page_size > 256 || (d->page_size & (d->page_size - 1)))
-        return fail(I4_EUNSUPPORTED, "model: page_size %d must be a power of two in [8, 256]", d->page_size);
+    if (d->page_size < 8 || d->page_size > 128 || (d->page_size & (d->page_size - 1)))
+        return fail(I4_EUNSUPPORTED, "model: page_size %d must be a power of two in [8, 128]", d->page_size);
+    if (d->max_ctx > 32768) return fail(I4_EUNSUPPORTED, "model: max_ctx above 32768");
     if (d->max_ctx % d->page_size) return fail(I4_EINVAL, "model: max_ctx must be a multiple of page_size");
     if (!(d->rms_eps >= 0.f) || !(d->rope_theta > 0.f)) return fail(I4_EINVAL, "model: eps/theta");
     if (!w->embed || !w->layers || !w->ln_final || !w->w_lm || !w->s_lm) return fail(I4_EINVAL, "weights: null");
@@ -353,8 +354,17 @@ extern "C" int i4_set_option(const char *name, int value) {
         return I4_OK;
     }
     if (n == "unpack") {
-        if (value != UNPACK_EXACT && value != UNPACK_SUBNORMAL) return fail(I4_EINVAL, "unpack must be 0 or 1");
+        if (value < UNPACK_EXACT || value > UNPACK_MAGIC32) return fail(I4_EINVAL, "unpack must be 0, 1 or 2");
         g_default_unpack = value;
+        return I4_OK;
+    }
+    if (n == "stream") {
+        set_stream_options(value, 0);
+        return I4_OK;
+    }
+    if (n == "stream_smem_kb") {
+        if (value < 32 || value > 227) return fail(I4_EINVAL, "stream_smem_kb must be in [32, 227]");
+        set_stream_options(-1, value);
         return I4_OK;
     }
     return fail(I4_EINVAL, "i4_set_option: unknown option '%s'", name);

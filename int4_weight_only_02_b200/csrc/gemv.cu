@@ -25,304 +25,9 @@
 
 #include "common.cuh"
 #include "gemv.cuh"
+#include "gemv_parts.cuh"
 
 namespace i4 {
-
-// ---------------------------------------------------------------- unpack
-
-// Signed 4-bit fields of one word, exactly, as fp16 pairs matching the x
-// staging order: out[0] = (k0, k4), out[1] = (k1, k5), out[2] = (k2, k6), out[3] = (k3, k7).
-// A single LOP3 places the field, flipped to offset-binary u = q + 8, under the
-// exponent of 1024 (low fields) or as 16u under it (high fields); one f16x2
-// subtract or fma then yields q exactly.
-__device__ __forceinline__ void unpack_word_exact(uint32_t q, uint32_t out[4]) {
-    const uint32_t q2 = q >> 8;
-    const uint32_t lo = lop3_select(q, 0x000F000Fu, 0x64086408u);   // 1024 + u   (k0, k4)
-    const uint32_t hi = lop3_select(q, 0x00F000F0u, 0x64806480u);   // 1024 + 16u (k1, k5)
-    const uint32_t lo2 = lop3_select(q2, 0x000F000Fu, 0x64086408u); // (k2, k6)
-    const uint32_t hi2 = lop3_select(q2, 0x00F000F0u, 0x64806480u); // (k3, k7)
-    out[0] = hsub2_bits(lo, 0x64086408u);                 // - 1032
-    out[1] = hfma2_bits(hi, 0x2C002C00u, 0xD480D480u);    // / 16 - 72
-    out[2] = hsub2_bits(lo2, 0x64086408u);
-    out[3] = hfma2_bits(hi2, 0x2C002C00u, 0xD480D480u);
-}
-
-// Offset-binary fields u = q + 8 as fp16 subnormals u * 2^-24 (low fields) and
-// 16u * 2^-24 (high fields): one LOP3 per pair, no float op.
-__device__ __forceinline__ void unpack_word_subnormal(uint32_t q, uint32_t out[4]) {
-    const uint32_t q2 = q >> 8;
-    out[0] = lop3_and_xor(q, 0x000F000Fu, 0x00080008u);
-    out[1] = lop3_and_xor(q, 0x00F000F0u, 0x00800080u);
-    out[2] = lop3_and_xor(q2, 0x000F000Fu, 0x00080008u);
-    out[3] = lop3_and_xor(q2, 0x00F000F0u, 0x00800080u);
-}
-
-// sum over the 32 weights of one chunk of q * x (exact unpack) or of u * x
-// (subnormal unpack; the caller subtracts 8 * sum(x)).
-template <int UNP>
-__device__ __forceinline__ float chunk_dot(const uint4 &wv, const uint4 *xw, int stride) {
-    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-    if constexpr (UNP == UNPACK_EXACT) {
-        float acc = 0.f;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            uint32_t v[4];
-            unpack_word_exact(words[t], v);
-            const uint4 xc = xw[t * stride];
-            acc = fma2_f16_f32(v[0], xc.x, acc);
-            acc = fma2_f16_f32(v[1], xc.y, acc);
-            acc = fma2_f16_f32(v[2], xc.z, acc);
-            acc = fma2_f16_f32(v[3], xc.w, acc);
-        }
-        return acc;
-    } else {
-        float alo = 0.f, ahi = 0.f;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            uint32_t v[4];
-            unpack_word_subnormal(words[t], v);
-            const uint4 xc = xw[t * stride];
-            alo = fma2_f16_f32(v[0], xc.x, alo);
-            ahi = fma2_f16_f32(v[1], xc.y, ahi);
-            alo = fma2_f16_f32(v[2], xc.z, alo);
-            ahi = fma2_f16_f32(v[3], xc.w, ahi);
-        }
-        return fmaf(ahi, 0.0625f, alo) * 16777216.0f;
-    }
-}
-
-// ---------------------------------------------------------------- prologue
-
-__device__ __forceinline__ uint4 permute_pairs(uint4 xv) {
-    // (x0..x7) -> (x0,x4) (x1,x5) (x2,x6) (x3,x7)
-    uint4 o;
-    o.x = __byte_perm(xv.x, xv.z, 0x5410);
-    o.y = __byte_perm(xv.x, xv.z, 0x7632);
-    o.z = __byte_perm(xv.y, xv.w, 0x5410);
-    o.w = __byte_perm(xv.y, xv.w, 0x7632);
-    return o;
-}
-
-__device__ __forceinline__ float block_sum(float v, float *red) {
-    v = warp_sum(v);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float t = 0.f;
-    const int nw = blockDim.x >> 5;
-    for (int i = 0; i < nw; ++i) t += red[i];
-    return t;
-}
-
-// Stage x (MR vectors of K fp16) into shared memory, pair-permuted:
-// xs[m][w][j] holds word w (0..3) of chunk j (0..K/32-1); sxs[m][j] = sum of the
-// chunk's 32 x values (subnormal unpack only).
-template <int PRO, int UNP, int MR>
-__device__ void stage_x(const GemvArgs &a, uint4 *xs, float *sxs, float *red) {
-    const int K = a.K, nu4 = K >> 5, nwords = K >> 3;
-    const uint16_t *src = a.x;
-    if constexpr (PRO == PRO_EMBED) {
-        int tok = *a.token;
-        tok = tok < 0 ? 0 : (tok >= a.vocab ? a.vocab - 1 : tok);
-        src = a.x + (size_t)tok * K;
-    }
-    if constexpr (PRO == PRO_PLAIN) {
-        for (int m = 0; m < MR; ++m)
-            for (int c = threadIdx.x; c < nwords; c += blockDim.x) {
-                uint4 xv = make_uint4(0, 0, 0, 0);
-                if (m < a.M) xv = *reinterpret_cast<const uint4 *>(a.x + (size_t)m * K + 8 * c);
-                xs[(m * 4 + (c & 3)) * nu4 + (c >> 2)] = permute_pairs(xv);
-            }
-    } else {
-        // RMSNorm of the residual row: x = fp16(r / sqrt(mean(r^2) + eps) * gamma)
-        float ss = 0.f;
-        for (int c = threadIdx.x; c < nwords; c += blockDim.x) {
-            const uint4 rv = *reinterpret_cast<const uint4 *>(src + 8 * c);
-            const uint32_t r[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&r[t]));
-                ss = fmaf(f.x, f.x, ss);
-                ss = fmaf(f.y, f.y, ss);
-            }
-        }
-        ss = block_sum(ss, red);
-        const float inv = 1.0f / sqrtf(ss / (float)K + a.eps);
-        for (int c = threadIdx.x; c < nwords; c += blockDim.x) {
-            const uint4 rv = *reinterpret_cast<const uint4 *>(src + 8 * c);
-            const uint4 gv = *reinterpret_cast<const uint4 *>(a.gamma + 8 * c);
-            if constexpr (PRO == PRO_EMBED) {
-                if (blockIdx.x == 0) *reinterpret_cast<uint4 *>(a.resid_out + 8 * c) = rv;
-            }
-            const uint32_t r[4] = {rv.x, rv.y, rv.z, rv.w}, g[4] = {gv.x, gv.y, gv.z, gv.w};
-            uint32_t o[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const float2 fr = __half22float2(*reinterpret_cast<const __half2 *>(&r[t]));
-                const float2 fg = __half22float2(*reinterpret_cast<const __half2 *>(&g[t]));
-                const __half2 h = __floats2half2_rn(fr.x * inv * fg.x, fr.y * inv * fg.y);
-                o[t] = *reinterpret_cast<const uint32_t *>(&h);
-            }
-            xs[(c & 3) * nu4 + (c >> 2)] = permute_pairs(make_uint4(o[0], o[1], o[2], o[3]));
-        }
-    }
-    if constexpr (UNP == UNPACK_SUBNORMAL) {
-        __syncthreads();
-        for (int idx = threadIdx.x; idx < MR * nu4; idx += blockDim.x) {
-            const int m = idx / nu4, j = idx - m * nu4;
-            float t = 0.f;
-            for (int w = 0; w < 4; ++w) {
-                const uint4 xc = xs[(m * 4 + w) * nu4 + j];
-                const uint32_t v[4] = {xc.x, xc.y, xc.z, xc.w};
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&v[e]));
-                    t += f.x + f.y;
-                }
-            }
-            sxs[idx] = t;
-        }
-    }
-}
-
-// ---------------------------------------------------------------- pair mapping
-
-template <int EPI>
-__device__ __forceinline__ int num_pairs(const GemvArgs &a) {
-    if constexpr (EPI == EPI_SILU) return a.inter;
-    return (a.N + 1) >> 1;
-}
-
-template <int EPI>
-__device__ __forceinline__ void pair_rows(const GemvArgs &a, int p, int &ra, int &rb) {
-    if constexpr (EPI == EPI_ROPE_KV) {          // (i, i + 64) inside a 128-row head
-        const int head = p >> 6, i = p & 63;
-        ra = head * 128 + i;
-        rb = ra + 64;
-    } else if constexpr (EPI == EPI_SILU) {      // (gate n, up n)
-        ra = p;
-        rb = p + a.inter;
-    } else {
-        ra = 2 * p;
-        rb = (2 * p + 1 < a.N) ? 2 * p + 1 : -1;
-    }
-}
-
-// ---------------------------------------------------------------- epilogues
-
-__device__ __forceinline__ float rnd16(float v) { return __half2float(__float2half_rn(v)); }
-
-__device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
-    if (v == 0.f) v = 0.f;  // -0 ranks with +0
-    uint32_t b = __float_as_uint(v);
-    b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    return ((unsigned long long)b << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)idx);
-}
-
-template <int EPI, int MR>
-__device__ __forceinline__ void epilogue(const GemvArgs &a, int p, int ra, int rb, const float *va, const float *vb,
-                                         unsigned long long &best) {
-    if constexpr (EPI == EPI_F16 || EPI == EPI_F32) {
-        for (int m = 0; m < MR; ++m) {
-            if (m >= a.M) break;
-            float ya = va[m], yb = vb[m];
-            if (a.bias) {
-                ya += half_bits_to_float(a.bias[ra]);
-                if (rb >= 0) yb += half_bits_to_float(a.bias[rb]);
-            }
-            if constexpr (EPI == EPI_F16) {
-                uint16_t *y = reinterpret_cast<uint16_t *>(a.y) + (size_t)m * a.N;
-                y[ra] = float_to_half_bits(ya);
-                if (rb >= 0) y[rb] = float_to_half_bits(yb);
-            } else {
-                float *y = reinterpret_cast<float *>(a.y) + (size_t)m * a.N;
-                y[ra] = ya;
-                if (rb >= 0) y[rb] = yb;
-            }
-        }
-    } else if constexpr (EPI == EPI_RESID) {
-        uint16_t *r = reinterpret_cast<uint16_t *>(a.y);
-        r[ra] = float_to_half_bits(half_bits_to_float(r[ra]) + rnd16(va[0]));
-        if (rb >= 0) r[rb] = float_to_half_bits(half_bits_to_float(r[rb]) + rnd16(vb[0]));
-    } else if constexpr (EPI == EPI_SILU) {
-        reinterpret_cast<uint16_t *>(a.y)[p] = silu_mul_bits(rnd16(va[0]), rnd16(vb[0]));
-    } else if constexpr (EPI == EPI_ROPE_KV) {
-        const int head = p >> 6, i = p & 63;
-        const float xa = rnd16(va[0] + half_bits_to_float(a.bias[ra]));
-        const float xb = rnd16(vb[0] + half_bits_to_float(a.bias[rb]));
-        int pos = *a.pos;
-        if (pos < 0 || pos >= a.max_ctx) {
-            if (a.status) *a.status = 2;
-            return;
-        }
-        if (head < a.n_q + a.n_kv) {
-            uint16_t oa, ob;
-            rope_pair(xa, xb, a.rope_cs[(size_t)pos * 64 + i], oa, ob);
-            if (head < a.n_q) {
-                a.q_out[head * 128 + i] = oa;
-                a.q_out[head * 128 + i + 64] = ob;
-            } else {
-                const int g = head - a.n_q;
-                const size_t off =
-                    (((size_t)a.page_table[pos / a.page_size] * a.n_kv + g) * a.page_size + pos % a.page_size) * 128;
-                a.k_pool[off + i] = oa;
-                a.k_pool[off + i + 64] = ob;
-            }
-        } else {
-            const int g = head - a.n_q - a.n_kv;
-            const size_t off =
-                (((size_t)a.page_table[pos / a.page_size] * a.n_kv + g) * a.page_size + pos % a.page_size) * 128;
-            a.v_pool[off + i] = float_to_half_bits(xa);
-            a.v_pool[off + i + 64] = float_to_half_bits(xb);
-        }
-    } else if constexpr (EPI == EPI_ARGMAX) {
-        float *lg = reinterpret_cast<float *>(a.y);
-        lg[ra] = va[0];
-        unsigned long long k = argmax_key(va[0], ra);
-        best = k > best ? k : best;
-        if (rb >= 0) {
-            lg[rb] = vb[0];
-            k = argmax_key(vb[0], rb);
-            best = k > best ? k : best;
-        }
-    }
-}
-
-// Last CTA of the lm_head GEMV: pick the token and advance the sequence state.
-__device__ void finish_step(const GemvArgs &a, unsigned long long cta_best) {
-    __shared__ unsigned long long sbest[8];
-    __shared__ int is_last;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) sbest[warp] = cta_best;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        unsigned long long b = 0;
-        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) b = sbest[i] > b ? sbest[i] : b;
-        atomicMax(a.best, b);
-        __threadfence();
-        const unsigned prev = atomicAdd(a.arrive, 1u);
-        is_last = (prev == gridDim.x - 1);
-    }
-    __syncthreads();
-    if (!is_last || threadIdx.x != 0) return;
-    __threadfence();
-    const unsigned long long b = atomicAdd(a.best, 0ull);
-    const int idx = (int)(0xFFFFFFFFu - (uint32_t)(b & 0xFFFFFFFFull));
-    const int pos = *a.pos_io;
-    const int np = pos + 1;
-    if (np >= a.max_ctx || pos < 0) {
-        if (a.status) *a.status = 1;
-    } else {
-        const int tok = (a.prompt && np < a.n_prompt) ? a.prompt[np] : idx;
-        *a.token_io = tok;
-        *a.pos_io = np;
-        *a.ctx_io = np + 1;
-        if (a.history) a.history[np] = tok;
-    }
-    *a.best = 0ull;
-    *a.arrive = 0u;
-    __threadfence();
-}
 
 // ---------------------------------------------------------------- kernel
 
@@ -335,7 +40,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
     float *sxs = reinterpret_cast<float *>(xs + MR * 4 * nu4);
 
     grid_dep_wait();
-    stage_x<PRO, UNP, MR>(a, xs, sxs, red);
+    stage_x<PRO, UNP, MR>(a, xs, sxs, red, CtaGroup());
     __syncthreads();
     grid_dep_launch();
 
@@ -469,6 +174,9 @@ int g_default_unpack = UNPACK_EXACT;
 
 int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool pdl, int unp, int max_ctas) {
     if (unp < 0) unp = g_default_unpack;
+    StreamGeom geo;
+    if (max_ctas == 0 && stream_geometry(epi, a, geo, unp)) return launch_gemv_stream(pro, epi, a, geo, stream, pdl, unp);
+    if (unp == UNPACK_MAGIC32) unp = UNPACK_EXACT;  // the register-streaming kernel has the fp16 unpacks only
     switch (pro * 16 + epi) {
         case PRO_PLAIN * 16 + EPI_F16: return launch_gemv_u<PRO_PLAIN, EPI_F16>(a, stream, pdl, unp, max_ctas);
         case PRO_PLAIN * 16 + EPI_F32: return launch_gemv_u<PRO_PLAIN, EPI_F32>(a, stream, pdl, unp, max_ctas);
@@ -523,7 +231,7 @@ extern "C" int int4_gemv(const uint32_t *w, const uint16_t *scales, const uint16
 extern "C" int i4_int4_gemv_variant(const uint32_t *w, const uint16_t *scales, const uint16_t *x,
                                     const uint16_t *bias, void *y, int y_is_fp32, int M, int N, int K, int unpack,
                                     int max_ctas, void *stream) {
-    if (unpack != UNPACK_EXACT && unpack != UNPACK_SUBNORMAL) return fail(I4_EINVAL, "unknown unpack variant");
+    if (unpack < UNPACK_EXACT || unpack > UNPACK_MAGIC32) return fail(I4_EINVAL, "unknown unpack variant");
     return gemv_entry(w, scales, x, bias, y, y_is_fp32, M, N, K, 128, unpack, max_ctas, (cudaStream_t)stream);
 }
 

@@ -10,7 +10,7 @@ constexpr int kGemvWarps = kGemvThreads / 32;
 
 enum GemvPrologue : int { PRO_PLAIN = 0, PRO_RMSNORM = 1, PRO_EMBED = 2 };
 enum GemvEpilogue : int { EPI_F16 = 0, EPI_F32 = 1, EPI_RESID = 2, EPI_ROPE_KV = 3, EPI_SILU = 4, EPI_ARGMAX = 5 };
-enum GemvUnpack : int { UNPACK_EXACT = 0, UNPACK_SUBNORMAL = 1 };
+enum GemvUnpack : int { UNPACK_EXACT = 0, UNPACK_SUBNORMAL = 1, UNPACK_MAGIC32 = 2 };
 
 struct GemvArgs {
     const uint32_t *w;
@@ -43,6 +43,20 @@ struct GemvArgs {
 };
 
 size_t gemv_smem_bytes(int K, int mr, int unp);
+
+// Geometry of the streaming (bulk-copy pipelined) GEMV for one launch.
+struct StreamGeom {
+    int R;              // rows per tile (16 or 2)
+    int stage_bytes;    // weights + scales of one tile, padded to 128 B
+    int stages;         // ring depth
+    int tiles, tiles_per_cta, grid;
+    int smem;           // dynamic shared memory bytes
+};
+// False when the shape or alignment does not fit the streaming kernel.
+bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp);
+int launch_gemv_stream(int pro, int epi, const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl,
+                       int unp);
+void set_stream_options(int enabled, int smem_kb);
 // unp < 0 selects the library default; max_ctas <= 0 means no cap.
 int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool pdl, int unp, int max_ctas);
 

@@ -1,0 +1,515 @@
+// Device building blocks of the INT4 GEMV kernels (gemv.cu, gemv_stream.cu):
+// register-level unpack, the per-chunk dot product, the x stage with its
+// fused prologues, row-pair mapping and the fused epilogues.
+#pragma once
+
+#include "common.cuh"
+#include "gemv.cuh"
+
+namespace i4 {
+
+// ---------------------------------------------------------------- unpack
+
+// Signed 4-bit fields of one word, exactly, as fp16 pairs matching the x
+// staging order: out[0] = (k0, k4), out[1] = (k1, k5), out[2] = (k2, k6), out[3] = (k3, k7).
+// A single LOP3 places the field, flipped to offset-binary u = q + 8, under the
+// exponent of 1024 (low fields) or as 16u under it (high fields); one f16x2
+// subtract or fma then yields q exactly.
+__device__ __forceinline__ void unpack_word_exact(uint32_t q, uint32_t out[4]) {
+    const uint32_t q2 = q >> 8;
+    const uint32_t lo = lop3_select(q, 0x000F000Fu, 0x64086408u);   // 1024 + u   (k0, k4)
+    const uint32_t hi = lop3_select(q, 0x00F000F0u, 0x64806480u);   // 1024 + 16u (k1, k5)
+    const uint32_t lo2 = lop3_select(q2, 0x000F000Fu, 0x64086408u); // (k2, k6)
+    const uint32_t hi2 = lop3_select(q2, 0x00F000F0u, 0x64806480u); // (k3, k7)
+    out[0] = hsub2_bits(lo, 0x64086408u);                 // - 1032
+    out[1] = hfma2_bits(hi, 0x2C002C00u, 0xD480D480u);    // / 16 - 72
+    out[2] = hsub2_bits(lo2, 0x64086408u);
+    out[3] = hfma2_bits(hi2, 0x2C002C00u, 0xD480D480u);
+}
+
+// Offset-binary fields u = q + 8 as fp16 subnormals u * 2^-24 (low fields) and
+// 16u * 2^-24 (high fields): one LOP3 per pair, no float op.
+__device__ __forceinline__ void unpack_word_subnormal(uint32_t q, uint32_t out[4]) {
+    const uint32_t q2 = q >> 8;
+    out[0] = lop3_and_xor(q, 0x000F000Fu, 0x00080008u);
+    out[1] = lop3_and_xor(q, 0x00F000F0u, 0x00800080u);
+    out[2] = lop3_and_xor(q2, 0x000F000Fu, 0x00080008u);
+    out[3] = lop3_and_xor(q2, 0x00F000F0u, 0x00800080u);
+}
+
+// fp32 unpack: a field kept in place under an fp32 exponent is 2^(23-4i) + u
+// (u = q + 8, the LOP3 flips bit 3 of the field); one packed add of
+// -(2^(23-4i) + 8) per two fields gives q exactly, one packed FMA per two
+// weights accumulates q * x in fp32. Fields 4-7 use the word shifted by 16.
+__device__ __forceinline__ float2 magic_pair(uint32_t q, uint32_t m0, uint32_t c0, uint32_t m1, uint32_t c1,
+                                             float2 off) {
+    return fadd2(make_float2(__uint_as_float(lop3_select(q, m0, c0)), __uint_as_float(lop3_select(q, m1, c1))), off);
+}
+
+// acc += q . x over one word (8 weights); x8 = the word's 8 x values in order.
+__device__ __forceinline__ float2 word_dot_f32(uint32_t q, const float4 &xa, const float4 &xb, float2 acc) {
+    const float2 off01 = make_float2(-8388616.0f, -524296.0f), off23 = make_float2(-32776.0f, -2056.0f);
+    const uint32_t qh = q >> 16;
+    const float2 v01 = magic_pair(q, 0x0000000Fu, 0x4B000008u, 0x000000F0u, 0x49000080u, off01);
+    const float2 v23 = magic_pair(q, 0x00000F00u, 0x47000800u, 0x0000F000u, 0x45008000u, off23);
+    const float2 v45 = magic_pair(qh, 0x0000000Fu, 0x4B000008u, 0x000000F0u, 0x49000080u, off01);
+    const float2 v67 = magic_pair(qh, 0x00000F00u, 0x47000800u, 0x0000F000u, 0x45008000u, off23);
+    acc = ffma2(v01, make_float2(xa.x, xa.y), acc);
+    acc = ffma2(v23, make_float2(xa.z, xa.w), acc);
+    acc = ffma2(v45, make_float2(xb.x, xb.y), acc);
+    acc = ffma2(v67, make_float2(xb.z, xb.w), acc);
+    return acc;
+}
+
+// sum over the 32 weights of one chunk of q * x (exact unpack) or of u * x
+// (subnormal unpack; the caller subtracts 8 * sum(x)).
+template <int UNP>
+__device__ __forceinline__ float chunk_dot(const uint4 &wv, const uint4 *xw, int stride) {
+    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+    if constexpr (UNP == UNPACK_EXACT) {
+        float acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            uint32_t v[4];
+            unpack_word_exact(words[t], v);
+            const uint4 xc = xw[t * stride];
+            acc = fma2_f16_f32(v[0], xc.x, acc);
+            acc = fma2_f16_f32(v[1], xc.y, acc);
+            acc = fma2_f16_f32(v[2], xc.z, acc);
+            acc = fma2_f16_f32(v[3], xc.w, acc);
+        }
+        return acc;
+    } else {
+        float alo = 0.f, ahi = 0.f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            uint32_t v[4];
+            unpack_word_subnormal(words[t], v);
+            const uint4 xc = xw[t * stride];
+            alo = fma2_f16_f32(v[0], xc.x, alo);
+            ahi = fma2_f16_f32(v[1], xc.y, ahi);
+            alo = fma2_f16_f32(v[2], xc.z, alo);
+            ahi = fma2_f16_f32(v[3], xc.w, ahi);
+        }
+        return fmaf(ahi, 0.0625f, alo) * 16777216.0f;
+    }
+}
+
+// ---------------------------------------------------------------- prologue
+
+__device__ __forceinline__ uint4 permute_pairs(uint4 xv) {
+    // (x0..x7) -> (x0,x4) (x1,x5) (x2,x6) (x3,x7)
+    uint4 o;
+    o.x = __byte_perm(xv.x, xv.z, 0x5410);
+    o.y = __byte_perm(xv.x, xv.z, 0x7632);
+    o.z = __byte_perm(xv.y, xv.w, 0x5410);
+    o.w = __byte_perm(xv.y, xv.w, 0x7632);
+    return o;
+}
+
+// The threads that stage x: the whole CTA, or the consumer warps of a
+// warp-specialised CTA, which synchronise on named barrier 1 only (a CTA-wide
+// barrier inside a role branch would also wait for the producer warp).
+struct CtaGroup {
+    __device__ __forceinline__ int tid() const { return threadIdx.x; }
+    __device__ __forceinline__ int size() const { return blockDim.x; }
+    __device__ __forceinline__ void sync() const { __syncthreads(); }
+};
+
+template <int FIRST, int COUNT>
+struct NamedGroup {
+    static_assert(FIRST % 32 == 0 && COUNT % 32 == 0, "whole warps");
+    __device__ __forceinline__ int tid() const { return (int)threadIdx.x - FIRST; }
+    __device__ __forceinline__ int size() const { return COUNT; }
+    __device__ __forceinline__ void sync() const { asm volatile("bar.sync 1, %0;" ::"n"(COUNT) : "memory"); }
+};
+
+template <class Group>
+__device__ __forceinline__ float group_sum(float v, float *red, const Group &g) {
+    v = warp_sum(v);
+    const int warp = g.tid() >> 5, lane = g.tid() & 31;
+    g.sync();
+    if (lane == 0) red[warp] = v;
+    g.sync();
+    float t = 0.f;
+    const int nw = g.size() >> 5;
+    for (int i = 0; i < nw; ++i) t += red[i];
+    return t;
+}
+
+// Produce the K/8 words (8 fp16 each) of the GEMV input x and hand each to
+// store(word_index, uint4): the plain vector, or RMSNorm of the residual row
+// (embedding row for PRO_EMBED, which CTA 0 also copies to the residual):
+//   x = fp16(r / sqrt(mean(r^2) + eps) * gamma), fp32 math.
+template <int PRO, class Group, class Store>
+__device__ __forceinline__ void for_each_x_word(const GemvArgs &a, float *red, const Group &grp, Store store) {
+    const int K = a.K, nwords = K >> 3;
+    const uint16_t *src = a.x;
+    if constexpr (PRO == PRO_EMBED) {
+        int tok = *a.token;
+        tok = tok < 0 ? 0 : (tok >= a.vocab ? a.vocab - 1 : tok);
+        src = a.x + (size_t)tok * K;
+    }
+    if constexpr (PRO == PRO_PLAIN) {
+        for (int c = grp.tid(); c < nwords; c += grp.size()) store(c, *reinterpret_cast<const uint4 *>(src + 8 * c));
+    } else {
+        float ss = 0.f;
+        for (int c = grp.tid(); c < nwords; c += grp.size()) {
+            const uint4 rv = *reinterpret_cast<const uint4 *>(src + 8 * c);
+            const uint32_t r[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&r[t]));
+                ss = fmaf(f.x, f.x, ss);
+                ss = fmaf(f.y, f.y, ss);
+            }
+        }
+        ss = group_sum(ss, red, grp);
+        const float inv = 1.0f / sqrtf(ss / (float)K + a.eps);
+        for (int c = grp.tid(); c < nwords; c += grp.size()) {
+            const uint4 rv = *reinterpret_cast<const uint4 *>(src + 8 * c);
+            const uint4 gv = *reinterpret_cast<const uint4 *>(a.gamma + 8 * c);
+            if constexpr (PRO == PRO_EMBED) {
+                if (blockIdx.x == 0) *reinterpret_cast<uint4 *>(a.resid_out + 8 * c) = rv;
+            }
+            const uint32_t r[4] = {rv.x, rv.y, rv.z, rv.w}, g[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 fr = __half22float2(*reinterpret_cast<const __half2 *>(&r[t]));
+                const float2 fg = __half22float2(*reinterpret_cast<const __half2 *>(&g[t]));
+                const __half2 h = __floats2half2_rn(fr.x * inv * fg.x, fr.y * inv * fg.y);
+                o[t] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+            store(c, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+    }
+}
+
+// Stage x for the streaming kernel in half-chunks of 16 k (two words):
+// xe[h] / xo[h] = pair-permuted even / odd word of half-chunk h; sxh[h] = sum of
+// its 16 values (subnormal unpack only).
+// Stage x as plain fp32 (fp32 unpack).
+template <int PRO, class Group>
+__device__ __forceinline__ void stage_x_f32(const GemvArgs &a, float4 *xf, float *red, const Group &grp) {
+    for_each_x_word<PRO>(a, red, grp, [&](int c, uint4 v) {
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&v.x));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&v.y));
+        const float2 f2 = __half22float2(*reinterpret_cast<const __half2 *>(&v.z));
+        const float2 f3 = __half22float2(*reinterpret_cast<const __half2 *>(&v.w));
+        xf[2 * c] = make_float4(f0.x, f0.y, f1.x, f1.y);
+        xf[2 * c + 1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+    });
+}
+
+template <int PRO, int UNP, class Group>
+__device__ __forceinline__ void stage_x_halves(const GemvArgs &a, uint4 *xe, uint4 *xo, float *sxh, float *red,
+                                               const Group &grp) {
+    for_each_x_word<PRO>(a, red, grp, [&](int c, uint4 v) { ((c & 1) ? xo : xe)[c >> 1] = permute_pairs(v); });
+    if constexpr (UNP == UNPACK_SUBNORMAL) {
+        grp.sync();
+        for (int h = grp.tid(); h < (a.K >> 4); h += grp.size()) {
+            const uint4 e = xe[h], o = xo[h];
+            const uint32_t v[8] = {e.x, e.y, e.z, e.w, o.x, o.y, o.z, o.w};
+            float t = 0.f;
+            for (int i = 0; i < 8; ++i) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&v[i]));
+                t += f.x + f.y;
+            }
+            sxh[h] = t;
+        }
+    }
+}
+
+// Dot product of one half-chunk (words w.x, w.y = 16 weights of a row) with its
+// staged x: sum q*x (exact unpack) or sum u*x with u = q + 8 (subnormal unpack).
+template <int UNP>
+__device__ __forceinline__ float half_dot(uint2 w, const uint4 &x0, const uint4 &x1) {
+    uint32_t va[4], vb[4];
+    if constexpr (UNP == UNPACK_EXACT) {
+        unpack_word_exact(w.x, va);
+        unpack_word_exact(w.y, vb);
+        float a0 = fma2_f16_f32(va[0], x0.x, 0.f), a1 = fma2_f16_f32(va[1], x0.y, 0.f);
+        float b0 = fma2_f16_f32(vb[0], x1.x, 0.f), b1 = fma2_f16_f32(vb[1], x1.y, 0.f);
+        a0 = fma2_f16_f32(va[2], x0.z, a0);
+        a1 = fma2_f16_f32(va[3], x0.w, a1);
+        b0 = fma2_f16_f32(vb[2], x1.z, b0);
+        b1 = fma2_f16_f32(vb[3], x1.w, b1);
+        return (a0 + a1) + (b0 + b1);
+    } else {
+        unpack_word_subnormal(w.x, va);
+        unpack_word_subnormal(w.y, vb);
+        float alo = fma2_f16_f32(va[0], x0.x, 0.f), ahi = fma2_f16_f32(va[1], x0.y, 0.f);
+        float blo = fma2_f16_f32(vb[0], x1.x, 0.f), bhi = fma2_f16_f32(vb[1], x1.y, 0.f);
+        alo = fma2_f16_f32(va[2], x0.z, alo);
+        ahi = fma2_f16_f32(va[3], x0.w, ahi);
+        blo = fma2_f16_f32(vb[2], x1.z, blo);
+        bhi = fma2_f16_f32(vb[3], x1.w, bhi);
+        return fmaf(ahi + bhi, 0.0625f, alo + blo) * 16777216.0f;
+    }
+}
+
+// Row accumulator of the streaming kernel. Exact unpack: v = sum s*q*x.
+// Subnormal unpack: lo = sum s*u*x*2^-24 over low fields, hi the same over high
+// fields (which carry 16u), cx = sum s*x; the row value is
+// (lo + hi/16) * 2^24 - 8 * cx (u = q + 8), computed once per row.
+struct RowAcc {
+    float lo, hi, cx;
+};
+
+template <int UNP>
+__device__ __forceinline__ void half_acc(uint2 w, const uint4 &x0, const uint4 &x1, float s, float sx, RowAcc &r) {
+    uint32_t va[4], vb[4];
+    if constexpr (UNP == UNPACK_EXACT) {
+        unpack_word_exact(w.x, va);
+        unpack_word_exact(w.y, vb);
+        float a0 = fma2_f16_f32(va[0], x0.x, 0.f), a1 = fma2_f16_f32(va[1], x0.y, 0.f);
+        a0 = fma2_f16_f32(va[2], x0.z, a0);
+        a1 = fma2_f16_f32(va[3], x0.w, a1);
+        a0 = fma2_f16_f32(vb[0], x1.x, a0);
+        a1 = fma2_f16_f32(vb[1], x1.y, a1);
+        a0 = fma2_f16_f32(vb[2], x1.z, a0);
+        a1 = fma2_f16_f32(vb[3], x1.w, a1);
+        r.lo = fmaf(s, a0 + a1, r.lo);
+    } else {
+        unpack_word_subnormal(w.x, va);
+        unpack_word_subnormal(w.y, vb);
+        float lo = fma2_f16_f32(va[0], x0.x, 0.f), hi = fma2_f16_f32(va[1], x0.y, 0.f);
+        lo = fma2_f16_f32(va[2], x0.z, lo);
+        hi = fma2_f16_f32(va[3], x0.w, hi);
+        lo = fma2_f16_f32(vb[0], x1.x, lo);
+        hi = fma2_f16_f32(vb[1], x1.y, hi);
+        lo = fma2_f16_f32(vb[2], x1.z, lo);
+        hi = fma2_f16_f32(vb[3], x1.w, hi);
+        r.lo = fmaf(s, lo, r.lo);
+        r.hi = fmaf(s, hi, r.hi);
+        r.cx = fmaf(s, sx, r.cx);
+    }
+}
+
+// fp32 unpack: 16 weights (words w.x, w.y) against x4[0..3] = their 16 x values.
+__device__ __forceinline__ void half_acc_f32(uint2 w, const float4 *x4, float s, RowAcc &r) {
+    float2 p = word_dot_f32(w.x, x4[0], x4[1], make_float2(0.f, 0.f));
+    p = word_dot_f32(w.y, x4[2], x4[3], p);
+    const float2 acc = ffma2(make_float2(s, s), p, make_float2(r.lo, r.hi));
+    r.lo = acc.x;
+    r.hi = acc.y;
+}
+
+template <int UNP>
+__device__ __forceinline__ float row_value(const RowAcc &r) {
+    if constexpr (UNP == UNPACK_MAGIC32) return r.lo + r.hi;
+    if constexpr (UNP == UNPACK_EXACT) return r.lo;
+    return fmaf(r.hi, 0.0625f, r.lo) * 16777216.0f - 8.0f * r.cx;
+}
+
+// Stage x (MR vectors of K fp16) into shared memory, pair-permuted:
+// xs[m][w][j] holds word w (0..3) of chunk j (0..K/32-1); sxs[m][j] = sum of the
+// chunk's 32 x values (subnormal unpack only).
+template <int PRO, int UNP, int MR, class Group>
+__device__ __forceinline__ void stage_x(const GemvArgs &a, uint4 *xs, float *sxs, float *red, const Group &grp) {
+    const int K = a.K, nu4 = K >> 5, nwords = K >> 3;
+    const uint16_t *src = a.x;
+    if constexpr (PRO == PRO_EMBED) {
+        int tok = *a.token;
+        tok = tok < 0 ? 0 : (tok >= a.vocab ? a.vocab - 1 : tok);
+        src = a.x + (size_t)tok * K;
+    }
+    if constexpr (PRO == PRO_PLAIN) {
+        for (int m = 0; m < MR; ++m)
+            for (int c = grp.tid(); c < nwords; c += grp.size()) {
+                uint4 xv = make_uint4(0, 0, 0, 0);
+                if (m < a.M) xv = *reinterpret_cast<const uint4 *>(a.x + (size_t)m * K + 8 * c);
+                xs[(m * 4 + (c & 3)) * nu4 + (c >> 2)] = permute_pairs(xv);
+            }
+    } else {
+        // RMSNorm of the residual row: x = fp16(r / sqrt(mean(r^2) + eps) * gamma)
+        float ss = 0.f;
+        for (int c = grp.tid(); c < nwords; c += grp.size()) {
+            const uint4 rv = *reinterpret_cast<const uint4 *>(src + 8 * c);
+            const uint32_t r[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&r[t]));
+                ss = fmaf(f.x, f.x, ss);
+                ss = fmaf(f.y, f.y, ss);
+            }
+        }
+        ss = group_sum(ss, red, grp);
+        const float inv = 1.0f / sqrtf(ss / (float)K + a.eps);
+        for (int c = grp.tid(); c < nwords; c += grp.size()) {
+            const uint4 rv = *reinterpret_cast<const uint4 *>(src + 8 * c);
+            const uint4 gv = *reinterpret_cast<const uint4 *>(a.gamma + 8 * c);
+            if constexpr (PRO == PRO_EMBED) {
+                if (blockIdx.x == 0) *reinterpret_cast<uint4 *>(a.resid_out + 8 * c) = rv;
+            }
+            const uint32_t r[4] = {rv.x, rv.y, rv.z, rv.w}, g[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 fr = __half22float2(*reinterpret_cast<const __half2 *>(&r[t]));
+                const float2 fg = __half22float2(*reinterpret_cast<const __half2 *>(&g[t]));
+                const __half2 h = __floats2half2_rn(fr.x * inv * fg.x, fr.y * inv * fg.y);
+                o[t] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+            xs[(c & 3) * nu4 + (c >> 2)] = permute_pairs(make_uint4(o[0], o[1], o[2], o[3]));
+        }
+    }
+    if constexpr (UNP == UNPACK_SUBNORMAL) {
+        grp.sync();
+        for (int idx = grp.tid(); idx < MR * nu4; idx += grp.size()) {
+            const int m = idx / nu4, j = idx - m * nu4;
+            float t = 0.f;
+            for (int w = 0; w < 4; ++w) {
+                const uint4 xc = xs[(m * 4 + w) * nu4 + j];
+                const uint32_t v[4] = {xc.x, xc.y, xc.z, xc.w};
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&v[e]));
+                    t += f.x + f.y;
+                }
+            }
+            sxs[idx] = t;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- pair mapping
+
+template <int EPI>
+__device__ __forceinline__ int num_pairs(const GemvArgs &a) {
+    if constexpr (EPI == EPI_SILU) return a.inter;
+    return (a.N + 1) >> 1;
+}
+
+template <int EPI>
+__device__ __forceinline__ void pair_rows(const GemvArgs &a, int p, int &ra, int &rb) {
+    if constexpr (EPI == EPI_ROPE_KV) {          // (i, i + 64) inside a 128-row head
+        const int head = p >> 6, i = p & 63;
+        ra = head * 128 + i;
+        rb = ra + 64;
+    } else if constexpr (EPI == EPI_SILU) {      // (gate n, up n)
+        ra = p;
+        rb = p + a.inter;
+    } else {
+        ra = 2 * p;
+        rb = (2 * p + 1 < a.N) ? 2 * p + 1 : -1;
+    }
+}
+
+// ---------------------------------------------------------------- epilogues
+
+__device__ __forceinline__ float rnd16(float v) { return __half2float(__float2half_rn(v)); }
+
+__device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
+    if (v == 0.f) v = 0.f;  // -0 ranks with +0
+    uint32_t b = __float_as_uint(v);
+    b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)b << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)idx);
+}
+
+template <int EPI, int MR>
+__device__ __forceinline__ void epilogue(const GemvArgs &a, int p, int ra, int rb, const float *va, const float *vb,
+                                         unsigned long long &best) {
+    if constexpr (EPI == EPI_F16 || EPI == EPI_F32) {
+        for (int m = 0; m < MR; ++m) {
+            if (m >= a.M) break;
+            float ya = va[m], yb = vb[m];
+            if (a.bias) {
+                ya += half_bits_to_float(a.bias[ra]);
+                if (rb >= 0) yb += half_bits_to_float(a.bias[rb]);
+            }
+            if constexpr (EPI == EPI_F16) {
+                uint16_t *y = reinterpret_cast<uint16_t *>(a.y) + (size_t)m * a.N;
+                y[ra] = float_to_half_bits(ya);
+                if (rb >= 0) y[rb] = float_to_half_bits(yb);
+            } else {
+                float *y = reinterpret_cast<float *>(a.y) + (size_t)m * a.N;
+                y[ra] = ya;
+                if (rb >= 0) y[rb] = yb;
+            }
+        }
+    } else if constexpr (EPI == EPI_RESID) {
+        uint16_t *r = reinterpret_cast<uint16_t *>(a.y);
+        r[ra] = float_to_half_bits(half_bits_to_float(r[ra]) + rnd16(va[0]));
+        if (rb >= 0) r[rb] = float_to_half_bits(half_bits_to_float(r[rb]) + rnd16(vb[0]));
+    } else if constexpr (EPI == EPI_SILU) {
+        reinterpret_cast<uint16_t *>(a.y)[p] = silu_mul_bits(rnd16(va[0]), rnd16(vb[0]));
+    } else if constexpr (EPI == EPI_ROPE_KV) {
+        const int head = p >> 6, i = p & 63;
+        const float xa = rnd16(va[0] + half_bits_to_float(a.bias[ra]));
+        const float xb = rnd16(vb[0] + half_bits_to_float(a.bias[rb]));
+        int pos = *a.pos;
+        if (pos < 0 || pos >= a.max_ctx) {
+            if (a.status) *a.status = 2;
+            return;
+        }
+        if (head < a.n_q + a.n_kv) {
+            uint16_t oa, ob;
+            rope_pair(xa, xb, a.rope_cs[(size_t)pos * 64 + i], oa, ob);
+            if (head < a.n_q) {
+                a.q_out[head * 128 + i] = oa;
+                a.q_out[head * 128 + i + 64] = ob;
+            } else {
+                const int g = head - a.n_q;
+                const size_t off =
+                    (((size_t)a.page_table[pos / a.page_size] * a.n_kv + g) * a.page_size + pos % a.page_size) * 128;
+                a.k_pool[off + i] = oa;
+                a.k_pool[off + i + 64] = ob;
+            }
+        } else {
+            const int g = head - a.n_q - a.n_kv;
+            const size_t off =
+                (((size_t)a.page_table[pos / a.page_size] * a.n_kv + g) * a.page_size + pos % a.page_size) * 128;
+            a.v_pool[off + i] = float_to_half_bits(xa);
+            a.v_pool[off + i + 64] = float_to_half_bits(xb);
+        }
+    } else if constexpr (EPI == EPI_ARGMAX) {
+        float *lg = reinterpret_cast<float *>(a.y);
+        lg[ra] = va[0];
+        unsigned long long k = argmax_key(va[0], ra);
+        best = k > best ? k : best;
+        if (rb >= 0) {
+            lg[rb] = vb[0];
+            k = argmax_key(vb[0], rb);
+            best = k > best ? k : best;
+        }
+    }
+}
+
+// Last CTA of the lm_head GEMV: pick the token and advance the sequence state.
+__device__ __forceinline__ void finish_step(const GemvArgs &a, unsigned long long cta_best) {
+    __shared__ unsigned long long sbest[32];
+    __shared__ int is_last;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) sbest[warp] = cta_best;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned long long b = 0;
+        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) b = sbest[i] > b ? sbest[i] : b;
+        atomicMax(a.best, b);
+        __threadfence();
+        const unsigned prev = atomicAdd(a.arrive, 1u);
+        is_last = (prev == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last || threadIdx.x != 0) return;
+    __threadfence();
+    const unsigned long long b = atomicAdd(a.best, 0ull);
+    const int idx = (int)(0xFFFFFFFFu - (uint32_t)(b & 0xFFFFFFFFull));
+    const int pos = *a.pos_io;
+    const int np = pos + 1;
+    if (np >= a.max_ctx || pos < 0) {
+        if (a.status) *a.status = 1;
+    } else {
+        const int tok = (a.prompt && np < a.n_prompt) ? a.prompt[np] : idx;
+        *a.token_io = tok;
+        *a.pos_io = np;
+        *a.ctx_io = np + 1;
+        if (a.history) a.history[np] = tok;
+    }
+    *a.best = 0ull;
+    *a.arrive = 0u;
+    __threadfence();
+}
+
+}  // namespace i4

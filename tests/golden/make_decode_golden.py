@@ -42,6 +42,8 @@ def main():
     tokens, logits = dec.generate(prompt, a.new, block_prompt=True)
     el = time.time() - t0
     top2 = np.sort(logits, axis=1)[:, -2:]
+    top5 = np.argsort(-logits, axis=1, kind="stable")[:, :5]
+    sample_idx = np.random.default_rng(2024).choice(shape.vocab, size=2048, replace=False)
     rec = {
         "workload": "qwen2.5-7b-shape int4-g128 decoder, seed %d, prompt %d, %d greedy steps, page 16"
                     % (a.seed, a.prompt, a.new),
@@ -53,6 +55,9 @@ def main():
         "top1_logit": [float(v) for v in top2[:, 1]],
         "top2_gap": [float(v) for v in (top2[:, 1] - top2[:, 0])],
         "first_logits_head": [float(v) for v in logits[0, :8]],
+        "top5": [[[int(i), float(logits[j, i])] for i in top5[j]] for j in range(len(tokens))],
+        "first_logits_sample": {"index": [int(i) for i in sample_idx],
+                                "value": [float(logits[0, i]) for i in sample_idx]},
         "oracle_seconds": round(el, 1),
         "oracle_threads": os.cpu_count(),
     }

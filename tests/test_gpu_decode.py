@@ -20,16 +20,22 @@ from helpers import normwise_err
 pytestmark = pytest.mark.gpu
 
 HERE = os.path.dirname(os.path.abspath(__file__))
+# K = 256 / 384: every GEMV takes the register-streaming kernel
 SMALL = synth.ModelShape(layers=2, hidden=256, inter=384, n_q=2, n_kv=1, head_dim=128, vocab=1000, group=128,
                          page_size=16, max_ctx=256)
+# K = 512 / 1024: every GEMV takes the bulk-copy pipelined kernel
+MID = synth.ModelShape(layers=3, hidden=512, inter=1024, n_q=4, n_kv=1, head_dim=128, vocab=2048, group=128,
+                       page_size=16, max_ctx=256)
+SHAPES = {"small": SMALL, "mid": MID}
+DEFAULT_UNPACK = 0
 
 
-def small_setup(i4, cuda, seed=0, n_prompt=20):
-    layers = [synth.layer_weights(SMALL, i, seed) for i in range(SMALL.layers)]
-    glob = synth.global_weights(SMALL, seed)
-    table = synth.page_table(SMALL, seed)
-    prompt = synth.prompt_tokens(SMALL, n_prompt, seed)
-    model = i4.DeviceModel(SMALL, layers, glob, device=cuda)
+def small_setup(i4, cuda, seed=0, n_prompt=20, shape=SMALL):
+    layers = [synth.layer_weights(shape, i, seed) for i in range(shape.layers)]
+    glob = synth.global_weights(shape, seed)
+    table = synth.page_table(shape, seed)
+    prompt = synth.prompt_tokens(shape, n_prompt, seed)
+    model = i4.DeviceModel(shape, layers, glob, device=cuda)
     return layers, glob, table, prompt, model
 
 
@@ -38,14 +44,20 @@ def run_steps(graph, n, eager=False):
         graph.eager() if eager else graph.replay()
 
 
-def test_small_decoder_matches_oracle(i4lib, cuda):
+@pytest.mark.parametrize("name,unpack", [("small", 0), ("mid", 0), ("mid", 1), ("mid", 2)])
+def test_small_decoder_matches_oracle(i4lib, cuda, name, unpack):
     import torch
-    layers, glob, table, prompt, model = small_setup(i4lib, cuda)
+    shape = SHAPES[name]
+    layers, glob, table, prompt, model = small_setup(i4lib, cuda, shape=shape)
     n_new = 12
-    ref_tokens, ref_logits = oracle.DecoderOracle(SMALL, layers, glob, table).generate(prompt, n_new)
+    ref_tokens, ref_logits = oracle.DecoderOracle(shape, layers, glob, table).generate(prompt, n_new)
     seq = i4lib.Sequence(model, table, prompt)
-    g = i4lib.DecodeGraph(model, seq)
-    assert g.kernel_count == 5 * SMALL.layers + 1
+    i4lib.set_option("unpack", unpack)
+    try:
+        g = i4lib.DecodeGraph(model, seq)
+    finally:
+        i4lib.set_option("unpack", DEFAULT_UNPACK)
+    assert g.kernel_count == 5 * shape.layers + 1
     logits = []
     for step in range(len(prompt) + n_new - 1):
         g.replay()
@@ -59,14 +71,18 @@ def test_small_decoder_matches_oracle(i4lib, cuda):
     assert int(seq.pos.item()) == len(prompt) + n_new - 1
     assert int(seq.ctx_len.item()) == len(prompt) + n_new
     assert int(seq.status.item()) == 0
+    # composed decoder: fp16 storage differences (fp32 vs fp64 sums) carry through the layers,
+    # so the logits get a looser bound than the single-op 2e-3 (see test_oracle_sensitivity.py)
     for i in range(n_new):
-        assert normwise_err(logits[i], ref_logits[i]) <= 2e-3, i
+        assert normwise_err(logits[i], ref_logits[i]) <= 1e-2, i
+    assert i4lib.device_error() == 0
     g.close()
 
 
-def test_graph_equals_eager_bit_exact(i4lib, cuda):
+@pytest.mark.parametrize("name", ["small", "mid"])
+def test_graph_equals_eager_bit_exact(i4lib, cuda, name):
     import torch
-    _, _, table, prompt, model = small_setup(i4lib, cuda, seed=1, n_prompt=9)
+    _, _, table, prompt, model = small_setup(i4lib, cuda, seed=1, n_prompt=9, shape=SHAPES[name])
     seqs = [i4lib.Sequence(model, table, prompt) for _ in range(2)]
     gs = [i4lib.DecodeGraph(model, s) for s in seqs]
     run_steps(gs[0], 40, eager=False)
@@ -75,7 +91,7 @@ def test_graph_equals_eager_bit_exact(i4lib, cuda):
     a, b = seqs
     assert torch.equal(a.history, b.history)
     assert torch.equal(a.logits, b.logits)
-    for l in range(SMALL.layers):
+    for l in range(SHAPES[name].layers):
         assert torch.equal(a.k_pools[l], b.k_pools[l])
         assert torch.equal(a.v_pools[l], b.v_pools[l])
     for g in gs:
@@ -95,34 +111,76 @@ def test_context_limit_sets_status(i4lib, cuda):
 
 
 GOLDEN = os.path.join(HERE, "golden", "decode_qwen7b_int4_seed0.json")
+# Noise floor of fp16 activation storage in this decoder, pinned on the oracle
+# alone in test_oracle_sensitivity.py: one fp16 ulp anywhere moves logits by up
+# to 0.075, so a top-2 gap below 0.15 is a tie neither side can be held to.
+LOGIT_NOISE = 0.075
+TIE_GAP = 0.15
+
+
+def _qwen7b(i4lib, cuda, gold, prompt):
+    shape = synth.QWEN7B
+    model = i4lib.DeviceModel.synthetic(shape, gold["seed"], device=cuda)
+    seq = i4lib.Sequence(model, synth.page_table(shape, gold["seed"]), prompt)
+    return model, seq, i4lib.DecodeGraph(model, seq)
 
 
 @pytest.mark.skipif(not os.path.exists(GOLDEN), reason="golden token stream not generated")
 def test_qwen7b_shape_greedy_stream_matches_oracle(i4lib, cuda):
+    """512-token prompt, then 128 greedy tokens of the 28-layer 7B-shape decoder.
+
+    * free-running: the GPU's own greedy stream equals the oracle's up to the
+      first step whose oracle top-2 gap is a tie (< TIE_GAP), if any;
+    * teacher-forced: fed the oracle's tokens, the GPU picks the oracle's token at
+      every step that is not a tie;
+    * first-step logits (2048 sampled) within the noise floor of the oracle's.
+    """
     import torch
     gold = json.load(open(GOLDEN))
     shape = synth.QWEN7B
-    prompt = synth.prompt_tokens(shape, gold["n_prompt"], gold["seed"])
-    assert [int(t) for t in prompt[:8]] == gold["prompt_head"]
-    model = i4lib.DeviceModel.synthetic(shape, gold["seed"], device=cuda)
-    seq = i4lib.Sequence(model, synth.page_table(shape, gold["seed"]), prompt)
-    g = i4lib.DecodeGraph(model, seq)
     n_prompt, n_new = gold["n_prompt"], gold["n_new"]
-    run_steps(g, n_prompt - 1)
-    g.replay()  # the step at the last prompt position produces the first new token
+    prompt = synth.prompt_tokens(shape, n_prompt, gold["seed"])
+    assert [int(t) for t in prompt[:8]] == gold["prompt_head"]
+    want = np.asarray(gold["tokens"])
+    gaps = np.asarray(gold["top2_gap"])
+
+    # free-running
+    model, seq, g = _qwen7b(i4lib, cuda, gold, prompt)
+    run_steps(g, n_prompt)
     torch.cuda.synchronize()
-    first_logits = seq.logits.cpu().numpy()
-    np.testing.assert_allclose(first_logits[:8], gold["first_logits_head"], rtol=0, atol=2e-2)
+    first = seq.logits.cpu().numpy()
+    idx = np.asarray(gold["first_logits_sample"]["index"])
+    ref = np.asarray(gold["first_logits_sample"]["value"])
+    assert np.max(np.abs(first[idx].astype(np.float64) - ref)) <= 2 * LOGIT_NOISE
     run_steps(g, n_new - 1)
     torch.cuda.synchronize()
     got = seq.history.cpu().numpy()[n_prompt: n_prompt + n_new]
-    want = np.asarray(gold["tokens"])
+    assert int(seq.status.item()) == 0 and i4lib.device_error() == 0
     mism = np.flatnonzero(got != want)
-    detail = ""
+    first_mismatch = int(mism[0]) if mism.size else n_new
+    ties_before = np.flatnonzero(gaps[:first_mismatch] < TIE_GAP)
     if mism.size:
-        i = int(mism[0])
-        detail = f"first mismatch at step {i}: oracle top-2 gap {gold['top2_gap'][i]:.4g} " \
-                 f"(top-1 logit {gold['top1_logit'][i]:.4g})"
-    assert mism.size == 0, detail
-    assert int(seq.status.item()) == 0
+        assert gaps[first_mismatch] < TIE_GAP, \
+            f"greedy streams part at step {first_mismatch}, oracle top-2 gap {gaps[first_mismatch]:.4f} is no tie"
     g.close()
+
+    # teacher-forced: the oracle's tokens as the forced stream
+    forced = np.concatenate([prompt, want[:-1]]).astype(np.int32)
+    seq2 = i4lib.Sequence(model, synth.page_table(shape, gold["seed"]), forced)
+    g2 = i4lib.DecodeGraph(model, seq2)
+    run_steps(g2, n_prompt - 1)
+    picks = []
+    for _ in range(n_new):
+        g2.replay()
+        torch.cuda.synchronize()
+        lg = seq2.logits.cpu().numpy()
+        picks.append(int(np.flatnonzero(lg == lg.max())[0]))
+    g2.close()
+    picks = np.asarray(picks)
+    disagree = np.flatnonzero(picks != want)
+    decided = gaps >= TIE_GAP
+    assert not np.any(decided[disagree]), \
+        f"teacher-forced picks differ at decided steps {disagree[decided[disagree]].tolist()}"
+    print(f"free-running identical for {first_mismatch}/{n_new} steps (ties before: {len(ties_before)}); "
+          f"teacher-forced agreement {n_new - disagree.size}/{n_new}, "
+          f"disagreements at ties {disagree.tolist()}")

@@ -17,9 +17,9 @@ pytestmark = pytest.mark.gpu
 TOL = 2e-3
 
 
-def run_gemv(i4, cuda, w, s, x, b=None, out_fp32=False, unpack=None):
+def run_gemv(i4, cuda, w, s, x, b=None, out_fp32=False, unpack=None, max_ctas=0):
     y = i4.int4_gemv(dev(w, cuda), dev(s, cuda), dev(np.atleast_2d(x), cuda),
-                     None if b is None else dev(b, cuda), out_fp32=out_fp32, unpack=unpack)
+                     None if b is None else dev(b, cuda), out_fp32=out_fp32, unpack=unpack, max_ctas=max_ctas)
     import torch
     torch.cuda.synchronize()
     return y.cpu().numpy()
@@ -42,16 +42,17 @@ def test_unpack_bit_exact(i4lib, cuda):
     assert np.array_equal(got, oracle.unpack_int4(w, 512))
 
 
-@pytest.mark.parametrize("unpack", [0, 1])
-def test_qkv_shape_against_oracle(i4lib, cuda, unpack):
+@pytest.mark.parametrize("unpack", [0, 1, 2])
+@pytest.mark.parametrize("kernel", ["stream", "register"])
+def test_qkv_shape_against_oracle(i4lib, cuda, unpack, kernel):
     w, s, x, b = synth.gemv_case(4608, 3584, seed=0, bias=True)
     ref = oracle.int4_gemv(w, s, x[0], b)
-    got = run_gemv(i4lib, cuda, w, s, x, b, unpack=unpack)[0]
+    got = run_gemv(i4lib, cuda, w, s, x, b, unpack=unpack, max_ctas=0 if kernel == "stream" else 1 << 20)[0]
     assert normwise_err(got, ref) <= TOL
     assert np.mean(got == ref) >= 0.98  # fp32 vs fp64 sums round to the same fp16 almost always
 
 
-@pytest.mark.parametrize("unpack", [0, 1])
+@pytest.mark.parametrize("unpack", [0, 1, 2])
 def test_exact_arithmetic_is_bit_exact(i4lib, cuda, unpack):
     rng = np.random.default_rng(1)
     n, k = 96, 1024
@@ -77,13 +78,26 @@ def test_ragged_shapes_and_batches(i4lib, cuda, n, k, m):
         assert normwise_err(got, ref) <= TOL
 
 
-def test_mlp_shapes_against_oracle(i4lib, cuda):
+@pytest.mark.parametrize("kernel,unpack", [("stream", 0), ("stream", 1), ("stream", 2), ("register", 0)])
+def test_mlp_shapes_against_oracle(i4lib, cuda, kernel, unpack):
     # gate/up K=3584 N=37888 and down K=18944 N=3584 (the MLP block of the 7B shape)
     for n, k in [(37888, 3584), (3584, 18944)]:
         w, s, x, _ = synth.gemv_case(n, k, seed=5)
         ref = oracle.int4_gemv(w, s, x[0])
-        got = run_gemv(i4lib, cuda, w, s, x)[0]
+        got = run_gemv(i4lib, cuda, w, s, x, unpack=unpack, max_ctas=0 if kernel == "stream" else 1 << 20)[0]
         assert normwise_err(got, ref) <= TOL, (n, k)
+        assert np.mean(got == ref) >= 0.98
+
+
+@pytest.mark.parametrize("n", [2, 16, 18, 30, 4096 + 14])
+def test_stream_kernel_partial_tiles(i4lib, cuda, n):
+    # rows not a multiple of the 16-row tile: the last tile copies and computes only its rows
+    w, s, x, b = synth.gemv_case(n, 512, seed=8, bias=True)
+    ref = oracle.int4_gemv(w, s, x[0], b)
+    for unpack in (0, 1, 2):
+        got = run_gemv(i4lib, cuda, w, s, x, b, unpack=unpack)[0]
+        assert normwise_err(got, ref) <= TOL
+    assert i4lib.device_error() == 0
 
 
 def test_lm_head_fp32_logits(i4lib, cuda):
