@@ -101,6 +101,30 @@ I4_API int paged_gqa_decode(const uint16_t *q, const uint16_t *k_pool, const uin
                      int max_pages_per_seq, float scale, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * paged_gqa_decode without a workspace argument and without any allocation.
+ * The pages have no counterpart of this call; it exists for callers that
+ * cannot hand out device memory: code that runs where cudaMalloc is not
+ * allowed or not wanted (inside a stream capture, on a real-time decode loop
+ * that must not block in the allocator, or as a plugin of a host framework
+ * that owns every device buffer).
+ *   Same arguments, layouts and results as paged_gqa_decode, minus ws and
+ *   ws_bytes. The split-K scratch is an 8 MiB array in the library's device
+ *   memory, which every GPU that loads the library keeps until the process
+ *   exits. A shape whose scratch (paged_gqa_decode_ws_bytes) exceeds 8 MiB is
+ *   rejected with I4_EUNSUPPORTED.
+ *   The first call on a device looks the array's address up (once per
+ *   device); make that first call before any stream capture.
+ *   Each call clears the merge counters with an asynchronous memset on
+ *   `stream`, then launches the kernel. All calls share the one array and it
+ *   keeps the last call's contents: calls that overlap on the GPU (for example
+ *   on two streams) race with each other. No cudaMalloc, cudaFree or other
+ *   allocating routine is called.
+ */
+I4_API int paged_gqa_decode_static(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_pool,
+                                   const int32_t *page_table, const int32_t *ctx_len, uint16_t *out, int B, int Hq,
+                                   int Hkv, int D, int page_size, int max_pages_per_seq, float scale, void *stream);
+
+/*
  * Test export: out[b][g][t][:] = pool row of token t (t < ctx_len[b]) for kv
  * head g, in token order (bit-exact page-indexing check). Rows t >= ctx_len[b]
  * are left untouched.  out [B][Hkv][max_ctx][D] fp16.

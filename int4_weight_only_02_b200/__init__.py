@@ -68,6 +68,7 @@ _SIGS = {
     "i4_int4_unpack": (_i, [_vp, _vp, _i, _i, _vp]),
     "paged_gqa_decode_ws_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "paged_gqa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
+    "paged_gqa_decode_static": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "i4_paged_gather": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "rmsnorm_rope": (_i, [ctypes.POINTER(RmsnormRopeArgs), _vp]),
     "i4_rmsnorm": (_i, [_vp, _vp, _vp, _vp, _i, _i, _f, _vp]),
@@ -179,6 +180,21 @@ def paged_gqa_decode(q, k_pool, v_pool, page_table, ctx_len, out=None, scale=Non
     _check(lib().paged_gqa_decode(_p(q), _p(k_pool), _p(v_pool), _p(page_table), _p(ctx_len), _p(out), B, Hq, Hkv, D,
                                   P, max_pages, float(scale), _p(ws), ws.numel() * ws.element_size(),
                                   _stream(stream)), "paged_gqa_decode")
+    return out
+
+
+def paged_gqa_decode_static(q, k_pool, v_pool, page_table, ctx_len, out=None, scale=None, stream=None):
+    """paged_gqa_decode with the library's fixed device scratch instead of a workspace (allocates nothing
+    besides `out` when it is not given)."""
+    import torch
+    B, Hq, D = q.shape
+    _, Hkv, P, _ = k_pool.shape
+    if out is None:
+        out = torch.empty_like(q)
+    scale = 1.0 / D ** 0.5 if scale is None else scale
+    _check(lib().paged_gqa_decode_static(_p(q), _p(k_pool), _p(v_pool), _p(page_table), _p(ctx_len), _p(out), B, Hq,
+                                         Hkv, D, P, page_table.shape[1], float(scale), _stream(stream)),
+           "paged_gqa_decode_static")
     return out
 
 

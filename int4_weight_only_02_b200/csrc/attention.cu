@@ -26,6 +26,8 @@
 // Pages below the current token's page were written by earlier decode steps,
 // so their copies start before the dependency wait (programmatic launch); the
 // page holding position ctx-1 is copied after it.
+#include <mutex>
+
 #include "async.cuh"
 #include "attention.cuh"
 #include "common.cuh"
@@ -401,6 +403,76 @@ extern "C" int paged_gqa_decode(const uint16_t *q, const uint16_t *k_pool, const
     p.scale = scale;
     p.splits = L.splits;
     p.ws = reinterpret_cast<char *>(ws);
+    p.counters_off = L.counters_off;
+    p.ml_off = L.ml_off;
+    p.acc_off = L.acc_off;
+    return launch_paged_gqa_decode(p, (cudaStream_t)stream, false);
+}
+
+// ---------------------------------------------------------------- no-allocation variant
+
+// Split-K scratch of paged_gqa_decode_static: a fixed array in the module's
+// device memory, so the call itself never allocates. Every GPU that loads the
+// library keeps these bytes until the process exits. All calls share it.
+static constexpr size_t kStaticScratchBytes = 8u << 20;
+static __device__ __align__(256) unsigned char g_attn_static_scratch[kStaticScratchBytes];
+
+static constexpr int kMaxDevices = 64;
+static std::mutex g_static_scratch_mu;
+static char *g_static_scratch_dev[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once per
+// device. The array's name in host code is only a host-side handle, never a
+// device address, so kernels get this pointer instead.
+static int static_scratch_ptr(char **out) {
+    int dev = 0;
+    int st = cuda_check(cudaGetDevice(&dev), "paged_gqa_decode_static: cudaGetDevice");
+    if (st) return st;
+    if (dev < 0 || dev >= kMaxDevices) return fail(I4_EUNSUPPORTED, "paged_gqa_decode_static: device %d", dev);
+    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+    if (!g_static_scratch_dev[dev]) {
+        void *ptr = nullptr;
+        st = cuda_check(cudaGetSymbolAddress(&ptr, g_attn_static_scratch), "paged_gqa_decode_static: scratch address");
+        if (st) return st;
+        g_static_scratch_dev[dev] = reinterpret_cast<char *>(ptr);
+    }
+    *out = g_static_scratch_dev[dev];
+    return I4_OK;
+}
+
+extern "C" int paged_gqa_decode_static(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_pool,
+                                       const int32_t *page_table, const int32_t *ctx_len, uint16_t *out, int B,
+                                       int Hq, int Hkv, int D, int page_size, int max_pages_per_seq, float scale,
+                                       void *stream) {
+    int st = attn_check(q, k_pool, v_pool, page_table, ctx_len, out, B, Hq, Hkv, D, page_size, max_pages_per_seq);
+    if (st) return st;
+    const AttnWs L = attn_ws_layout(B, Hq, Hkv, page_size, max_pages_per_seq);
+    if (L.bytes > kStaticScratchBytes)
+        return fail(I4_EUNSUPPORTED,
+                    "paged_gqa_decode_static: this shape needs %zu bytes of split-K scratch, the static scratch "
+                    "holds %zu; use paged_gqa_decode with a caller workspace",
+                    L.bytes, kStaticScratchBytes);
+    char *ws = nullptr;
+    if ((st = static_scratch_ptr(&ws))) return st;
+    // the merge counters must start at zero; the rest of the scratch is written before it is read
+    st = cuda_check(cudaMemsetAsync(ws + L.counters_off, 0, (size_t)B * Hkv * sizeof(unsigned), (cudaStream_t)stream),
+                    "paged_gqa_decode_static: clearing the counters");
+    if (st) return st;
+    AttnParams p = {};
+    p.q = q;
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.page_table = page_table;
+    p.ctx_len = ctx_len;
+    p.out = out;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.page_size = page_size;
+    p.max_pages = max_pages_per_seq;
+    p.scale = scale;
+    p.splits = L.splits;
+    p.ws = ws;
     p.counters_off = L.counters_off;
     p.ml_off = L.ml_off;
     p.acc_off = L.acc_off;
