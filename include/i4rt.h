@@ -261,7 +261,7 @@ I4_API int decode_step_launch_kernel(i4_graph *g, int index, void *stream);
 
 /*
  * Library options, applied to graphs created afterwards and to later calls:
- *   "pdl"    0/1: launch the kernels of a decode step with programmatic
+ *   "pdl"    0/1 (default 1): launch the kernels of a decode step with programmatic
  *            dependent launch (each kernel still waits for its predecessor's
  *            results before reading them);
  *   "unpack" 0/1: INT4 unpack variant of the GEMV (0 exact fp16 values,

@@ -28,7 +28,7 @@
 namespace i4 {
 int launch_rope_table(float2 *cs, int max_ctx, int d, double theta, cudaStream_t stream);
 bool g_dry_run = false;
-bool g_pdl = false;
+bool g_pdl = true;
 }  // namespace i4
 
 using namespace i4;

@@ -12,3 +12,14 @@ def normwise_err(got, ref):
 def dev(a, device):
     from int4_weight_only_02_b200.runtime import to_device
     return to_device(np.asarray(a), device)
+
+
+# Greedy-decode tie bound of the 28-layer 7B-shape decoder, derived on the oracle
+# alone (test_oracle_sensitivity.py): fp32 sums round about 1 % of fp16 stores
+# differently from fp64 sums; injecting such +-1-ulp flips at a 1 % rate into the
+# oracle moves the last-token logits by ~0.06-0.08 RMS (up to ~0.4) after a
+# 64-128 token context, so a top-2 gap below 3 * sqrt(2) * 0.07 ~= 0.3 is a tie
+# that neither implementation can be held to.
+FLIP_RATE = 0.01
+TIE_GAP = 0.3
+LOGIT_NOISE_MAX = 0.4
