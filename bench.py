@@ -124,7 +124,7 @@ def traffic_from_profile(kernel_src: str):
         return None
 
 
-def oracle_cpu_sample(shape, layers_np, glob_np, n_tokens: int = 2):
+def oracle_cpu_sample(shape, layers_np, glob_np, n_tokens: int = 8):
     """The CPU oracle as it stands: n_tokens decode steps at position 512 with the KV
     cache below it filled with random fp16 values."""
     import numpy as np
@@ -195,6 +195,55 @@ def run_reference(args):
     return 0
 
 
+def max_over_ranks(value_ms: float, world: int, device) -> float:
+    """The slowest rank's time (all ranks take part in the same collective)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(steps: int, world: int, ms_max: float) -> float:
+    """Replicas: every rank decodes `steps` tokens of its own sequence; the job rate uses the slowest rank."""
+    return world * steps / (ms_max / 1e3)
+
+
+PROFILE_KERNELS = {"qkv": 0, "attention": 1, "o": 2, "gate_up": 3, "down": 4, "lm_head": 5}
+
+
+def run_profile_kernel(args):
+    """One-layer decoder with the 7B layer shapes (1.5 GB on the device); launches one kernel of the
+    decode step `--launches` times. Not a benchmark: a small, fixed case for ncu."""
+    import torch
+
+    import int4_weight_only_02_b200 as i4
+    from int4_weight_only_02_b200 import synth
+    if args.pdl is not None:
+        i4.set_option("pdl", args.pdl)
+    if args.unpack is not None:
+        i4.set_option("unpack", args.unpack)
+    shape = synth.ModelShape(layers=1)
+    dev = torch.device("cuda", 0)
+    layers = [synth.layer_weights(synth.QWEN7B, 0, 0)]
+    glob = synth.global_weights(shape, 0)
+    model = i4.DeviceModel(shape, layers, glob, device=dev)
+    seq = i4.Sequence(model, synth.page_table(shape, 0), synth.prompt_tokens(shape, 512, 0))
+    graph = i4.DecodeGraph(model, seq)
+    for _ in range(args.prime_steps):
+        graph.replay()
+    k = PROFILE_KERNELS[args.profile_kernel]
+    index = k if k < 5 else graph.kernel_count - 1
+    for _ in range(args.launches):
+        graph.launch_kernel(index)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_kernel": args.profile_kernel, "index": index, "launches": args.launches,
+                      "device_error": i4.device_error()}))
+    graph.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -205,10 +254,17 @@ def main():
     ap.add_argument("--eager-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pdl", type=int, default=None, help="override programmatic dependent launch (0/1)")
-    ap.add_argument("--unpack", type=int, default=None, help="override the GEMV unpack variant (0/1)")
+    ap.add_argument("--unpack", type=int, default=None, help="override the GEMV unpack variant (0..3)")
+    ap.add_argument("--profile-kernel", default=None, choices=sorted(PROFILE_KERNELS),
+                    help="profiling mode: a one-layer model of the same shapes, then only this kernel of the "
+                         "decode step, --launches times (for ncu captures)")
+    ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--prime-steps", type=int, default=0, help="profiling mode: decode steps run first")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_kernel:
+        return run_profile_kernel(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
@@ -274,11 +330,7 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = ev0.elapsed_time(ev1)
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     ms_tok = ms_max / args.steps
     status = int(seq.status.item())
     ctx1 = int(seq.ctx_len.item())
@@ -300,10 +352,7 @@ def main():
         tok_h[0] = out_h[0]
     e1.record(stream)
     torch.cuda.synchronize()
-    t = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_tok_s = world * args.steps / (float(t.item()) / 1e3)
+    e2e_tok_s = job_tokens_per_s(args.steps, world, max_over_ranks(e0.elapsed_time(e1), world, dev))
 
     # eager launches of the same kernels (the pages' eager-vs-graph comparison)
     torch.cuda.synchronize()
@@ -315,20 +364,26 @@ def main():
     eager_ms = e0.elapsed_time(e1) / max(args.eager_steps, 1)
 
     # dominant kernel alone: RMSNorm + gate/up GEMV + SiLU of each layer (70 MB each, L2-cold)
-    def time_kernel(index_fn, reps=2):
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(shape.layers * reps)]
-        ends = [torch.cuda.Event(enable_timing=True) for _ in range(shape.layers * reps)]
+    def time_kernel(index_fn, reps=3):
+        """Mean device time of one launch: the kernel of every layer captured back to back in one
+        CUDA graph, replayed `reps` times between two events on the launching stream."""
+        side = torch.cuda.Stream()
+        cg = torch.cuda.CUDAGraph()
         torch.cuda.synchronize()
-        torch.cuda._sleep(100_000_000)  # keep the GPU busy while the host queues every launch
-        for r in range(reps):
-            for li in range(shape.layers):
-                j = r * shape.layers + li
-                starts[j].record(stream)
-                graph.launch_kernel(index_fn(li))
-                ends[j].record(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(cg, stream=side):
+                for li in range(shape.layers):
+                    graph.launch_kernel(index_fn(li))
         torch.cuda.synchronize()
-        d = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-        return statistics.mean(d[shape.layers:]) if reps > 1 else statistics.mean(d)
+        cg.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            cg.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * shape.layers)
 
     h, inter = shape.hidden, shape.inter
     gu_bytes = 2 * inter * (h // 2) + 2 * inter * (h // 128) * 2 + 2 * h * 2 + inter * 2
@@ -340,6 +395,7 @@ def main():
     qkv_ms = time_kernel(lambda li: 5 * li + 0)
     o_bytes = h * (h // 2) + h * (h // 128) * 2 + h * 2 + 2 * h * 2
     o_ms = time_kernel(lambda li: 5 * li + 2)
+    attn_ms = time_kernel(lambda li: 5 * li + 1)
     torch.cuda.synchronize()
     # restore a consistent residual/KV state is not needed afterwards: nothing else runs
 
@@ -354,7 +410,7 @@ def main():
     step_gbs = step_bytes / (ms_tok * 1e-3) / 1e9
 
     line = {
-        "metric": METRIC, "value": round(world * args.steps / (ms_max / 1e3), 2), "unit": "tok/s",
+        "metric": METRIC, "value": round(job_tokens_per_s(args.steps, world, ms_max), 2), "unit": "tok/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_tok, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
@@ -370,7 +426,9 @@ def main():
             "qkv": {"us": round(qkv_ms * 1e3, 2), "GBs": round(qkv_bytes / (qkv_ms * 1e-3) / 1e9, 1)},
             "o": {"us": round(o_ms * 1e3, 2), "GBs": round(o_bytes / (o_ms * 1e-3) / 1e9, 1)},
             "gate_up": {"us": round(gu_ms * 1e3, 2), "GBs": round(gu_gbs, 1)},
-            "down": {"us": round(down_ms * 1e3, 2), "GBs": round(down_bytes / (down_ms * 1e-3) / 1e9, 1)}},
+            "down": {"us": round(down_ms * 1e3, 2), "GBs": round(down_bytes / (down_ms * 1e-3) / 1e9, 1)},
+            "attention": {"us": round(attn_ms * 1e3, 2),
+                          "GBs": round(2 * shape.n_kv * shape.head_dim * 2 * (ctx1 - 1) / (attn_ms * 1e-3) / 1e9, 1)}},
         "step_roofline": {"bytes_per_step": int(step_bytes), "achieved_GBs": round(step_gbs, 1),
                           "frac_of_8TBs": round(step_gbs / NOMINAL_HBM_GBS, 4),
                           "frac_of_measured": round(step_gbs / peak, 4)},
@@ -379,6 +437,16 @@ def main():
         "gpu_launches": args.steps * n_k,
         "clocks": clocks.summary(),
     }
+    golden = os.path.join(ROOT, "tests", "golden", "decode_qwen7b_int4_seed0.json")
+    if rank == 0 and args.prompt == 512 and os.path.exists(golden):
+        gold = json.load(open(golden))
+        hist = seq.history.cpu().numpy()[512: 512 + len(gold["tokens"])]
+        n = min(len(hist), int(seq.pos.item()) + 1 - 512)
+        same = 0
+        while same < n and int(hist[same]) == int(gold["tokens"][same]):
+            same += 1
+        line["greedy_vs_oracle"] = {"compared": n, "identical_prefix": same,
+                                    "note": "free-running; first difference expected at an oracle top-2 near-tie"}
     graph.close()
     if world > 1:
         dist.barrier()

@@ -38,7 +38,7 @@ constexpr int kAttnThreads = 128;
 constexpr int kMaxGroup = 8;
 constexpr int kHeadDim = 128;
 constexpr int kMaxTokensPerSplit = 128;
-constexpr int kMinTokensPerSplit = 32;
+constexpr int kMinTokensPerSplit = 64;
 constexpr int kMaxSplits = 256;
 constexpr int kMaxCtx = kMaxSplits * kMaxTokensPerSplit;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
     __shared__ float sc[kMaxGroup][kMaxTokensPerSplit];
     __shared__ float red[4][kMaxGroup][kHeadDim];
     __shared__ float coef[kMaxGroup][kMaxSplits];
+    __shared__ float lsum[kMaxGroup][kMaxSplits];
     __shared__ float mh[kMaxGroup], lh[kMaxGroup];
     __shared__ __align__(8) uint64_t kbar, vbar;
     __shared__ int is_last;
@@ -280,25 +281,38 @@ __global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnPara
     if (!is_last) return;
     __threadfence();
 
-    if (tid < G) {
-        const int h = tid;
-        float M = -INFINITY;
-        for (int j = 0; j < active; ++j) M = fmaxf(M, __ldcg(&ml[cell0 + (size_t)j * G + h]).x);
-        float L = 0.f;
-        for (int j = 0; j < active; ++j) {
-            const float2 v = __ldcg(&ml[cell0 + (size_t)j * G + h]);
-            const float w = exp2f(v.x - M);
-            coef[h][j] = w;
-            L = fmaf(w, v.y, L);
+    // every split's (m, l) into shared memory at once (one coalesced pass), then per head
+    // (warp w takes heads w, w + 4) the maximum and the normalised weights 2^(m_j - M) / L
+    for (int i = tid; i < active * G; i += kAttnThreads) {
+        const float2 v = __ldcg(&ml[cell0 + i]);
+        coef[i % G][i / G] = v.x;
+        lsum[i % G][i / G] = v.y;
+    }
+    __syncthreads();
+    {
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int h = warp; h < G; h += 4) {
+            float M = -INFINITY;
+            for (int j = lane; j < active; j += 32) M = fmaxf(M, coef[h][j]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            float L = 0.f;
+            for (int j = lane; j < active; j += 32) {
+                const float w = exp2f(coef[h][j] - M);
+                coef[h][j] = w;
+                L = fmaf(w, lsum[h][j], L);
+            }
+            L = warp_sum(L);
+            const float invL = 1.0f / L;
+            __syncwarp();
+            for (int j = lane; j < active; j += 32) coef[h][j] *= invL;
         }
-        const float invL = 1.0f / L;
-        for (int j = 0; j < active; ++j) coef[h][j] *= invL;
     }
     __syncthreads();
     for (int i = tid; i < G * kHeadDim; i += kAttnThreads) {
         const int h = i / kHeadDim, d = i % kHeadDim;
         float o = 0.f;
-#pragma unroll 8
+#pragma unroll 16
         for (int j = 0; j < active; ++j) o = fmaf(coef[h][j], __ldcg(&pacc[(cell0 + (size_t)j * G + h) * kHeadDim + d]), o);
         p.out[((size_t)b * p.Hq + g * G + h) * kHeadDim + d] = float_to_half_bits(o);
     }

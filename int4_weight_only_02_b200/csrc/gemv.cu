@@ -176,7 +176,9 @@ int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool p
     if (unp < 0) unp = g_default_unpack;
     StreamGeom geo;
     if (max_ctas == 0 && stream_geometry(epi, a, geo, unp)) return launch_gemv_stream(pro, epi, a, geo, stream, pdl, unp);
-    if (unp == UNPACK_MAGIC32) unp = UNPACK_EXACT;  // the register-streaming kernel has the fp16 unpacks only
+    if (max_ctas == 0 && unp == UNPACK_MMA && stream_geometry(epi, a, geo, UNPACK_SUBNORMAL))
+        return launch_gemv_stream(pro, epi, a, geo, stream, pdl, UNPACK_SUBNORMAL);  // rows too long for 16-row tiles
+    if (unp == UNPACK_MAGIC32 || unp == UNPACK_MMA) unp = UNPACK_SUBNORMAL;  // register kernel: fp16 unpacks only
     switch (pro * 16 + epi) {
         case PRO_PLAIN * 16 + EPI_F16: return launch_gemv_u<PRO_PLAIN, EPI_F16>(a, stream, pdl, unp, max_ctas);
         case PRO_PLAIN * 16 + EPI_F32: return launch_gemv_u<PRO_PLAIN, EPI_F32>(a, stream, pdl, unp, max_ctas);
@@ -196,7 +198,8 @@ int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool p
 using namespace i4;
 
 static int gemv_entry(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
-                      int y_is_fp32, int M, int N, int K, int group, int unp, int max_ctas, cudaStream_t stream) {
+                      int y_is_fp32, int M, int N, int K, int group, int unp, int max_ctas, cudaStream_t stream,
+                      void *ws = nullptr, size_t ws_bytes = 0) {
     if (!w || !scales || !x || !y) return fail(I4_EINVAL, "int4_gemv: null pointer");
     if (group != 128) return fail(I4_EUNSUPPORTED, "int4_gemv: group must be 128 (got %d)", group);
     if (K <= 0 || K % 128 != 0 || K > 32768)
@@ -218,6 +221,15 @@ static int gemv_entry(const uint32_t *w, const uint16_t *scales, const uint16_t 
     a.M = M;
     a.bias = bias;
     a.y = y;
+    if (ws) {
+        const size_t need = ksplit_ws_bytes(N, K);
+        if (!need) return fail(I4_EUNSUPPORTED, "int4_gemv: no K-split kernel for K=%d", K);
+        if (ws_bytes < need || !aligned(ws, 256))
+            return fail(I4_EINVAL, "int4_gemv: K-split workspace of %zu bytes (256-aligned) needed", need);
+        const size_t cnt = ((size_t)(N + 15) / 16 * sizeof(unsigned) + 255) & ~(size_t)255;
+        a.tile_cnt = reinterpret_cast<unsigned *>(ws);
+        a.part_ws = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + cnt);
+    }
     return launch_gemv(PRO_PLAIN, y_is_fp32 ? EPI_F32 : EPI_F16, a, stream, false, unp, max_ctas);
 }
 
@@ -230,10 +242,13 @@ extern "C" int int4_gemv(const uint32_t *w, const uint16_t *scales, const uint16
 // (0 = none); used by the tests and the benchmark to compare variants.
 extern "C" int i4_int4_gemv_variant(const uint32_t *w, const uint16_t *scales, const uint16_t *x,
                                     const uint16_t *bias, void *y, int y_is_fp32, int M, int N, int K, int unpack,
-                                    int max_ctas, void *stream) {
-    if (unpack < UNPACK_EXACT || unpack > UNPACK_MAGIC32) return fail(I4_EINVAL, "unknown unpack variant");
-    return gemv_entry(w, scales, x, bias, y, y_is_fp32, M, N, K, 128, unpack, max_ctas, (cudaStream_t)stream);
+                                    int max_ctas, void *ws, size_t ws_bytes, void *stream) {
+    if (unpack < UNPACK_EXACT || unpack > UNPACK_MMA) return fail(I4_EINVAL, "unknown unpack variant");
+    return gemv_entry(w, scales, x, bias, y, y_is_fp32, M, N, K, 128, unpack, max_ctas, (cudaStream_t)stream, ws,
+                      ws_bytes);
 }
+
+extern "C" size_t i4_int4_gemv_ksplit_ws_bytes(int N, int K) { return N > 0 && K > 0 ? ksplit_ws_bytes(N, K) : 0; }
 
 extern "C" int i4_int4_unpack(const uint32_t *w, int8_t *q, int N, int K, void *stream) {
     if (!w || !q) return fail(I4_EINVAL, "i4_int4_unpack: null pointer");

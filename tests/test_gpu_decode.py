@@ -26,7 +26,10 @@ SMALL = synth.ModelShape(layers=2, hidden=256, inter=384, n_q=2, n_kv=1, head_di
 # K = 512 / 1024: every GEMV takes the bulk-copy pipelined kernel
 MID = synth.ModelShape(layers=3, hidden=512, inter=1024, n_q=4, n_kv=1, head_dim=128, vocab=2048, group=128,
                        page_size=16, max_ctx=256)
-SHAPES = {"small": SMALL, "mid": MID}
+# intermediate 4608 > 4096: the down projection takes the K-split tensor-core kernel (unpack 3)
+LONG = synth.ModelShape(layers=2, hidden=512, inter=4608, n_q=4, n_kv=1, head_dim=128, vocab=2048, group=128,
+                        page_size=16, max_ctx=256)
+SHAPES = {"small": SMALL, "mid": MID, "long": LONG}
 DEFAULT_UNPACK = 0
 
 
@@ -44,7 +47,8 @@ def run_steps(graph, n, eager=False):
         graph.eager() if eager else graph.replay()
 
 
-@pytest.mark.parametrize("name,unpack", [("small", 0), ("mid", 0), ("mid", 1), ("mid", 2)])
+@pytest.mark.parametrize("name,unpack", [("small", 0), ("mid", 0), ("mid", 1), ("mid", 2), ("mid", 3), ("long", 1),
+                                         ("long", 3)])
 def test_small_decoder_matches_oracle(i4lib, cuda, name, unpack):
     import torch
     shape = SHAPES[name]

@@ -42,7 +42,7 @@ def test_unpack_bit_exact(i4lib, cuda):
     assert np.array_equal(got, oracle.unpack_int4(w, 512))
 
 
-@pytest.mark.parametrize("unpack", [0, 1, 2])
+@pytest.mark.parametrize("unpack", [0, 1, 2, 3])
 @pytest.mark.parametrize("kernel", ["stream", "register"])
 def test_qkv_shape_against_oracle(i4lib, cuda, unpack, kernel):
     w, s, x, b = synth.gemv_case(4608, 3584, seed=0, bias=True)
@@ -52,7 +52,7 @@ def test_qkv_shape_against_oracle(i4lib, cuda, unpack, kernel):
     assert np.mean(got == ref) >= 0.98  # fp32 vs fp64 sums round to the same fp16 almost always
 
 
-@pytest.mark.parametrize("unpack", [0, 1, 2])
+@pytest.mark.parametrize("unpack", [0, 1, 2, 3])
 def test_exact_arithmetic_is_bit_exact(i4lib, cuda, unpack):
     rng = np.random.default_rng(1)
     n, k = 96, 1024
@@ -78,7 +78,7 @@ def test_ragged_shapes_and_batches(i4lib, cuda, n, k, m):
         assert normwise_err(got, ref) <= TOL
 
 
-@pytest.mark.parametrize("kernel,unpack", [("stream", 0), ("stream", 1), ("stream", 2), ("register", 0)])
+@pytest.mark.parametrize("kernel,unpack", [("stream", 0), ("stream", 1), ("stream", 2), ("stream", 3), ("register", 0)])
 def test_mlp_shapes_against_oracle(i4lib, cuda, kernel, unpack):
     # gate/up K=3584 N=37888 and down K=18944 N=3584 (the MLP block of the 7B shape)
     for n, k in [(37888, 3584), (3584, 18944)]:
@@ -94,7 +94,7 @@ def test_stream_kernel_partial_tiles(i4lib, cuda, n):
     # rows not a multiple of the 16-row tile: the last tile copies and computes only its rows
     w, s, x, b = synth.gemv_case(n, 512, seed=8, bias=True)
     ref = oracle.int4_gemv(w, s, x[0], b)
-    for unpack in (0, 1, 2):
+    for unpack in (0, 1, 2, 3):
         got = run_gemv(i4lib, cuda, w, s, x, b, unpack=unpack)[0]
         assert normwise_err(got, ref) <= TOL
     assert i4lib.device_error() == 0
@@ -118,3 +118,22 @@ def test_bad_arguments_raise(i4lib, cuda):
         i4lib.int4_gemv(wd, sd, xd, group=64)
     with pytest.raises(i4lib.I4Error):
         i4lib.int4_gemv(wd, sd, torch.zeros((9, 256), dtype=torch.float16, device=cuda))
+
+
+@pytest.mark.parametrize("n,k", [(3584, 18944), (64, 4608), (30, 8192)])
+def test_ksplit_tensor_core_kernel(i4lib, cuda, n, k):
+    """Rows too long for whole-row tiles: the K-split mma.sync kernel with its workspace."""
+    import torch
+    w, s, x, b = synth.gemv_case(n, k, seed=9, bias=True)
+    ref = oracle.int4_gemv(w, s, x[0], b)
+    nbytes = i4lib.int4_gemv_ksplit_ws_bytes(n, k)
+    assert nbytes > 0
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=cuda)
+    args = [dev(a, cuda) for a in (w, s, x)]
+    for _ in range(2):  # the counters must come back to zero for the second call
+        got = i4lib.int4_gemv(*args, bias=dev(b, cuda), unpack=3, ws=ws)
+        torch.cuda.synchronize()
+        assert normwise_err(got.cpu().numpy()[0], ref) <= TOL
+    cnt = ((n + 15) // 16 * 4 + 255) // 256 * 256
+    assert int(ws[:cnt].sum().item()) == 0
+    assert i4lib.device_error() == 0
