@@ -1,31 +1,38 @@
-// Paged grouped-query decode attention: split-K over KV pages with a
-// log-sum-exp merge.
+// Paged grouped-query decode attention: split-K over the context with a
+// log-sum-exp merge, on tensor cores.
 //
-// "How To Build Your Own LLM Runtime From Scratch" ("Technical Details":
-// paged KV cache and attention; lessons: a __syncthreads() inside a
+// "How To Build Your Own LLM Runtime From Scratch" ("Technical Details": paged
+// KV cache and attention; lessons: a __syncthreads() inside a
 // warp-specialised branch corrupted the softmax at KV-page tails). The H100
-// design there was warp-specialised with TMA; at batch 1 a decode head reads
-// well under 1 MB, so this kernel has no producer/consumer roles: thread 0
-// issues one bulk copy (cp.async.bulk, no multicast) per K page and per V page
-// of the CTA's range into shared memory, every thread then runs the same
-// three phases, and every barrier is reached by the whole CTA (CTAs without
-// work leave before the first barrier, as a whole).
+// design there was warp-specialised with TMA. At batch 1 one kv head of one
+// layer holds well under 1 MB of K/V at the contexts decode runs at, so this
+// kernel is bound by latency, not bandwidth, and its design keeps the chain
+// from launch to output short:
 //
-// Grid (S, Hkv, B). CTA (s, g, b) takes pages [s*pps, (s+1)*pps) of sequence b
-// for kv head g and all G = Hq/Hkv query heads that share it, so each K/V row
-// is read once for G heads. pps is derived on the device from ctx_len[b], so a
-// captured graph stays valid as the context grows. One page of one kv head is
-// page_size contiguous rows of 256 bytes, so a page is one copy.
-//   phase A: 16 threads per token (8 dims each), 8 tokens per pass;
-//            scores = q.k * scale * log2(e) into shared memory.
-//   phase B: per head, max and sum of exp2 over the CTA's tokens.
-//   phase C: o[h][:] += p[h][t] * V[t][:], same thread layout as phase A.
-// With one active split the CTA writes the normalised output; otherwise it
-// writes (m, l, o) partials and the last CTA to arrive for (b, g) merges them:
-//   M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
-// Pages below the current token's page were written by earlier decode steps,
-// so their copies start before the dependency wait (programmatic launch); the
-// page holding position ctx-1 is copied after it.
+//  * Work. Grid (S, Hkv, B) in clusters of CL CTAs along x. The context of
+//    sequence b is cut into tiles of 64 tokens and CTA s takes tiles
+//    [s*tpc, (s+1)*tpc). tpc comes from ctx_len[b] on the device, so a captured
+//    graph stays valid as the context grows; contexts of up to 2*CL tiles stay
+//    inside one cluster.
+//  * Data. A producer warp brings each tile's K and V rows into a two-stage
+//    shared-memory ring with 2-D TMA copies (one per page piece and 64-dim
+//    half, 128-byte swizzle, no multicast). A page below the one holding
+//    position ctx-1 was written by an earlier step, so its copy is issued before
+//    the programmatic dependency wait; the current page after it.
+//  * Math. Each of 4 consumer warps takes 16 tokens of a tile.
+//    S = Q K^T on mma.m16n8k16 with the G <= 8 query heads that share the kv
+//    head as the M rows (rows G..15 are zero), so each K row is read once for
+//    all G heads. P = 2^(S - m) rounded to fp16 then feeds O^T = V^T P^T
+//    (M = 16 dims, N = 8 heads, K = 16 tokens) directly from the S
+//    accumulators. Online softmax per warp, fp32 accumulation throughout.
+//  * Merge. The 4 warps merge in shared memory; the CTAs of a cluster push
+//    their (m, l, o) into the rank-0 CTA's shared memory (distributed shared
+//    memory), which merges them. With one active cluster that CTA writes the
+//    output; otherwise cluster leaders write partials to the workspace and the
+//    last to arrive merges them:
+//      M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+#include <cuda.h>  // CUtensorMap and its enums; the encoder is looked up in the driver at run time
+
 #include <mutex>
 
 #include "async.cuh"
@@ -34,305 +41,532 @@
 
 namespace i4 {
 
-constexpr int kAttnThreads = 128;
-constexpr int kMaxGroup = 8;
 constexpr int kHeadDim = 128;
-constexpr int kMaxTokensPerSplit = 128;
-constexpr int kMinTokensPerSplit = 64;
+constexpr int kMaxGroup = 8;                               // query heads per kv head (MMA rows used)
+constexpr int kWarpTokens = 16;                            // tokens of a tile per consumer warp
+constexpr int kConsumerWarps = 4;
+constexpr int kTileTokens = kConsumerWarps * kWarpTokens;  // 64
+constexpr int kStages = 2;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kAttnThreads = kConsumerThreads + 32;        // + the producer warp
+constexpr int kMaxCluster = 8;
+constexpr int kOneClusterTiles = 2;  // contexts up to kMaxCluster * this many tiles stay in one cluster
 constexpr int kMaxSplits = 256;
-constexpr int kMaxCtx = kMaxSplits * kMaxTokensPerSplit;
+constexpr int kMaxCtx = 32768;
+constexpr int kMaxPageSize = 128;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr unsigned long long kPoolRows = (1ull << 31) - 1;  // row bound of the pool tensor maps (rows are int32)
+
+// Dynamic shared memory, from a 1024-byte aligned base (128-byte swizzle atoms):
+//   ring  kStages x {K dims 0-63, K dims 64-127, V dims 0-63, V dims 64-127}, each [64 tokens][128 B]
+//   recv  [kMaxCluster][kHeadDim][kMaxGroup] fp32 o and [kMaxCluster][kMaxGroup] (m, l) pushed by the cluster
+// The warp partials reuse ring stage 0 once every tile is consumed; the cross-cluster merge reuses recv.
+constexpr unsigned kHalfBytes = kTileTokens * 128;
+constexpr unsigned kStageBytes = 4 * kHalfBytes;
+constexpr unsigned kRingBytes = kStages * kStageBytes;
+constexpr unsigned kRecvOff = kRingBytes;
+constexpr unsigned kRecvBytes = kMaxCluster * kHeadDim * kMaxGroup * 4;
+constexpr unsigned kRecvMlOff = kRecvOff + kRecvBytes;
+constexpr unsigned kDynSmem = 1024 + kRecvMlOff + kMaxCluster * kMaxGroup * 8;
+static_assert(kConsumerWarps * kHeadDim * kMaxGroup * 4 <= kStageBytes, "warp partials must fit in one stage");
+static_assert(2 * kMaxGroup * kMaxSplits * 4 <= kRecvBytes, "merge weights must fit in the receive buffer");
 
 __device__ int g_attn_error = 0;
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-int attn_splits(int B, int Hkv, int page_size, int max_pages) {
-    // enough CTAs to cover the SMs twice, no split above kMaxTokensPerSplit tokens
-    const int max_pps = kMaxTokensPerSplit / page_size > 0 ? kMaxTokensPerSplit / page_size : 1;
-    int s_min = (max_pages + max_pps - 1) / max_pps;
-    int s_par = (2 * kNumSMs + B * Hkv - 1) / (B * Hkv);
-    int s = s_par > s_min ? s_par : s_min;
-    if (s > max_pages) s = max_pages;
-    if (s > kMaxSplits) s = kMaxSplits;
-    return s < 1 ? 1 : s;
+// How the n_tiles tiles of one sequence are spread over the `splits` CTAs of a (b, g) row.
+struct Split {
+    int tpc, active, clusters;  // tiles per CTA, CTAs with tiles, clusters with such CTAs
+};
+__host__ __device__ inline Split split_work(int n_tiles, int splits, int cl) {
+    Split w;
+    w.tpc = n_tiles <= cl * kOneClusterTiles ? (n_tiles + cl - 1) / cl : (n_tiles + splits - 1) / splits;
+    if (w.tpc < 1) w.tpc = 1;
+    w.active = (n_tiles + w.tpc - 1) / w.tpc;
+    w.clusters = (w.active + cl - 1) / cl;
+    return w;
 }
 
 AttnWs attn_ws_layout(int B, int Hq, int Hkv, int page_size, int max_pages) {
+    // about two CTAs per SM over the grid, whole clusters, no more CTAs than tiles
+    const int max_tiles = (int)(((long long)max_pages * page_size + kTileTokens - 1) / kTileTokens);
+    const int rows = B * Hkv;
+    int s = (2 * kNumSMs + rows - 1) / rows;
+    s = s < max_tiles ? s : max_tiles;
+    s = s < kMaxSplits ? s : kMaxSplits;
+    s = s < 1 ? 1 : s;
+    const int cl = s < kMaxCluster ? s : kMaxCluster;
     AttnWs L;
-    L.splits = attn_splits(B, Hkv, page_size, max_pages);
+    L.splits = s / cl * cl;
+    L.cluster = cl;
     const size_t G = (size_t)(Hq / Hkv);
-    const size_t cells = (size_t)B * Hkv * L.splits * G;
+    const size_t cells = (size_t)rows * (L.splits / cl) * G;  // one partial per cluster and head
     L.counters_off = 0;
-    L.ml_off = align256((size_t)B * Hkv * sizeof(unsigned));
+    L.ml_off = align256((size_t)rows * sizeof(unsigned));
     L.acc_off = L.ml_off + align256(cells * sizeof(float2));
     L.bytes = L.acc_off + align256(cells * kHeadDim * sizeof(float));
     return L;
 }
 
-// Largest token range one CTA can be given: the shared-memory K and V tiles are this long.
-static int attn_tile_tokens(const AttnParams &p) {
-    const int min_pps = (kMinTokensPerSplit + p.page_size - 1) / p.page_size;
-    int pps = (p.max_pages + p.splits - 1) / p.splits;
-    pps = pps < min_pps ? min_pps : pps;
-    return pps * p.page_size;
+// ------------------------------------------------------------------ device helpers
+
+struct __align__(64) AttnMaps {
+    CUtensorMap k, v;  // [rows = pages*Hkv*P][128] fp16 views of the pools, box 64 dims x min(P, 64) rows
+};
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
 }
 
-__global__ void __launch_bounds__(kAttnThreads) paged_gqa_decode_kernel(AttnParams p) {
-    extern __shared__ __align__(128) unsigned char kv_smem[];
-    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int G = p.Hq / p.Hkv;
-    const int P = p.page_size;
-    const int max_ctx = p.max_pages * P;
-    int ctx = p.ctx_len[b];  // written by an earlier step, never by this kernel's predecessor
-    ctx = ctx < 1 ? 1 : (ctx > max_ctx ? max_ctx : ctx);
-    const int n_pages = (ctx + P - 1) / P;
-    const int min_pps = (kMinTokensPerSplit + P - 1) / P;
-    int pps = (n_pages + p.splits - 1) / p.splits;
-    pps = pps < min_pps ? min_pps : pps;
-    const int active = (n_pages + pps - 1) / pps;
-    if (s >= active) return;  // the whole CTA leaves; no barrier has been reached
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
 
-    __shared__ float qs[kMaxGroup][kHeadDim];
-    __shared__ float sc[kMaxGroup][kMaxTokensPerSplit];
-    __shared__ float red[4][kMaxGroup][kHeadDim];
-    __shared__ float coef[kMaxGroup][kMaxSplits];
-    __shared__ float lsum[kMaxGroup][kMaxSplits];
-    __shared__ float mh[kMaxGroup], lh[kMaxGroup];
-    __shared__ __align__(8) uint64_t kbar, vbar;
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// d += A(16x16, row) * B(16x8, col), fp16 inputs, fp32 accumulation
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory"); }
+__device__ __forceinline__ void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+__device__ __forceinline__ void st_cluster_f2(uint32_t addr, float a, float b) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory"); }
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+
+// weight of a partial with maximum m under the merged maximum M (0 for an empty partial)
+__device__ __forceinline__ float merge_weight(float m, float M) {
+    return m == -INFINITY ? 0.f : exp2f(m - (M == -INFINITY ? 0.f : M));
+}
+
+// ------------------------------------------------------------------ the kernel
+
+__global__ void __launch_bounds__(kAttnThreads, 2)
+    paged_gqa_decode_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
+    __shared__ float2 wml[kMaxCluster][kMaxGroup];  // (m, l) of the 4 warps, later of the cluster's CTAs
+    __shared__ float cw[kMaxCluster][kMaxGroup];    // merge weights
+    __shared__ float cM[kMaxGroup], cL[kMaxGroup];
     __shared__ int is_last;
 
-    const int tid = threadIdx.x;
-    const int p0 = s * pps;
-    const int p1 = (p0 + pps) < n_pages ? (p0 + pps) : n_pages;
-    const int t0 = p0 * P;
-    const int t1 = (p1 * P) < ctx ? (p1 * P) : ctx;
-    const int T = t1 - t0;
-    const int32_t *table = p.page_table + (size_t)b * p.max_pages;
-    const float qscale = p.scale * kLog2e;
-    const unsigned page_bytes = (unsigned)P * kHeadDim * 2;
-    unsigned char *ks = kv_smem;                                   // [tile tokens][128] fp16
-    unsigned char *vs = kv_smem + (size_t)p.tile_tokens * kHeadDim * 2;
-    const int last_page = n_pages - 1;                            // holds position ctx-1
+    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = p.Hq / p.Hkv, P = p.page_size, CL = p.cluster;
+    const int max_ctx = p.max_pages * P;
+    int ctx = p.ctx_len[b];  // advanced by an earlier step's last kernel, never by this kernel's predecessor
+    ctx = ctx < 1 ? 1 : (ctx > max_ctx ? max_ctx : ctx);
+    const int n_tiles = (ctx + kTileTokens - 1) / kTileTokens;
+    const Split w = split_work(n_tiles, p.splits, CL);
+    if (s / CL >= w.clusters) return;  // the whole cluster leaves before any barrier
+    cluster_arrive_relaxed();          // "started": awaited before the first store into the leader
+    const uint32_t rank = cluster_rank();
+    const int tile0 = s * w.tpc;
+    int n_my = n_tiles - tile0;
+    n_my = n_my < 0 ? 0 : (n_my > w.tpc ? w.tpc : n_my);
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char *gbase = smem_raw + (base - raw);
 
     if (tid == 0) {
-        mbar_init(&kbar, 1);
-        mbar_init(&vbar, 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kConsumerWarps);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    const uint64_t pol = evict_first_policy();
-    if (tid == 0) {
-        mbar_expect_tx(&kbar, (unsigned)(p1 - p0) * page_bytes);
-        mbar_expect_tx(&vbar, (unsigned)(p1 - p0) * page_bytes);
-        for (int pg = p0; pg < p1; ++pg) {
-            if (pg == last_page) continue;
-            const size_t off = ((size_t)table[pg] * p.Hkv + g) * P * kHeadDim;
-            bulk_load(ks + (size_t)(pg - p0) * page_bytes, p.k_pool + off, page_bytes, &kbar, pol);
-            bulk_load(vs + (size_t)(pg - p0) * page_bytes, p.v_pool + off, page_bytes, &vbar, pol);
-        }
-    }
-    grid_dep_wait();  // q and the current token's K/V row come from the preceding kernel
-    if (tid == 0 && last_page >= p0 && last_page < p1) {
-        const size_t off = ((size_t)table[last_page] * p.Hkv + g) * P * kHeadDim;
-        bulk_load(ks + (size_t)(last_page - p0) * page_bytes, p.k_pool + off, page_bytes, &kbar, pol);
-        bulk_load(vs + (size_t)(last_page - p0) * page_bytes, p.v_pool + off, page_bytes, &vbar, pol);
-    }
 
-    // q of the G heads, fp32, pre-scaled
-    for (int i = tid; i < G * kHeadDim; i += kAttnThreads) {
-        const int h = i / kHeadDim, d = i % kHeadDim;
-        qs[h][d] = half_bits_to_float(p.q[((size_t)b * p.Hq + g * G + h) * kHeadDim + d]) * qscale;
-    }
-    __syncthreads();
-    bool ok = mbar_wait(&kbar, 0);
-    if (!ok) record_error(&g_attn_error, 1);
-
-    const int tk = tid >> 4;         // token lane 0..7
-    const int dl = tid & 15;         // 8 dims [8dl, 8dl+8)
-    // ---- phase A: scores
-    {
-        float qr[kMaxGroup][8];
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) qr[h][e] = h < G ? qs[h][8 * dl + e] : 0.f;
-        // every lane runs the same passes (the shuffles below need the full warp)
-        for (int tb = 0; tb < T; tb += 8) {
-            const int t = tb + tk;
-            const bool live = t < T;
-            uint4 kv = make_uint4(0, 0, 0, 0);
-            if (live && ok) kv = *reinterpret_cast<const uint4 *>(ks + ((size_t)t * kHeadDim + 8 * dl) * 2);
-            const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-            float kf[8];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&kw[e]));
-                kf[2 * e] = f.x;
-                kf[2 * e + 1] = f.y;
+    if (warp == kConsumerWarps) {
+        // ---------------- producer: lane = piece * 4 + part (K lo, K hi, V lo, V hi)
+        const int R = P < kTileTokens ? P : kTileTokens;  // rows per copy: one page, or 64 rows of a larger page
+        const int pieces = kTileTokens / R;
+        const int last_page = (ctx - 1) / P;
+        const int32_t *table = p.page_table + (size_t)b * p.max_pages;
+        bool waited = false;
+        for (int i = 0; i < n_my; ++i) {
+            const int st = i % kStages, use = i / kStages;
+            if (use > 0 && !mbar_wait(&empty[st], (unsigned)((use - 1) & 1))) {
+                record_error(&g_attn_error, 1);
+                break;
             }
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h) {
-                float d = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) d = fmaf(qr[h][e], kf[e], d);
-#pragma unroll
-                for (int o = 8; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-                if (live && dl == 0 && h < G) sc[h][t] = d;
+            const int t0 = (tile0 + i) * kTileTokens;
+            int n_pc = (ctx - t0 + R - 1) / R;
+            n_pc = n_pc < pieces ? n_pc : pieces;
+            if (!waited && (t0 + n_pc * R - 1) / P >= last_page) {
+                grid_dep_wait();  // the current page's new row comes from the preceding kernel
+                asm volatile("fence.proxy.async;" ::: "memory");
+                waited = true;
+            }
+            if (lane == 0) mbar_expect_tx(&full[st], (unsigned)(n_pc * 4 * R * 128));
+            __syncwarp();
+            if (lane < n_pc * 4) {
+                const int pc = lane >> 2, part = lane & 3;
+                const int t = t0 + pc * R;
+                const int y = (table[t / P] * p.Hkv + g) * P + (t % P);
+                const uint32_t dst = base + st * kStageBytes + part * kHalfBytes + pc * R * 128;
+                tma_load_2d(dst, part < 2 ? &maps.k : &maps.v, (part & 1) * 64, y, &full[st]);
             }
         }
-    }
-    __syncthreads();
-
-    // ---- phase B: per-head max and sum of exp2 (warp w takes heads w, w+4)
-    {
-        const int warp = tid >> 5, lane = tid & 31;
-        for (int h = warp; h < G; h += 4) {
-            float m = -INFINITY;
-            for (int t = lane; t < T; t += 32) m = fmaxf(m, sc[h][t]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            float l = 0.f;
-            for (int t = lane; t < T; t += 32) {
-                const float e = exp2f(sc[h][t] - m);
-                sc[h][t] = e;
-                l += e;
-            }
-            l = warp_sum(l);
-            if (lane == 0) {
-                mh[h] = m;
-                lh[h] = l;
-            }
-        }
-    }
-    __syncthreads();
-    if (!mbar_wait(&vbar, 0)) {
-        record_error(&g_attn_error, 1);
-        ok = false;
-    }
-
-    // ---- phase C: o = sum_t p_t v_t
-    float acc[kMaxGroup][8];
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
-    for (int t = tk; t < T && ok; t += 8) {
-        const uint4 vv = *reinterpret_cast<const uint4 *>(vs + ((size_t)t * kHeadDim + 8 * dl) * 2);
-        const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
-        float vf[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&vw[e]));
-            vf[2 * e] = f.x;
-            vf[2 * e + 1] = f.y;
-        }
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            if (h < G) {
-                const float pt = sc[h][t];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(pt, vf[e], acc[h][e]);
-            }
-        }
-    }
-    // reduce the 8 token lanes: lanes l and l^16 share dims, then across the 4 warps
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], 16);
-    const int warp = tid >> 5;
-    if ((tid & 31) < 16) {
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h)
-            if (h < G)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) red[warp][h][8 * dl + e] = acc[h][e];
-    }
-    __syncthreads();
-
-    if (active == 1) {
-        for (int i = tid; i < G * kHeadDim; i += kAttnThreads) {
-            const int h = i / kHeadDim, d = i % kHeadDim;
-            const float o = (red[0][h][d] + red[1][h][d]) + (red[2][h][d] + red[3][h][d]);
-            p.out[((size_t)b * p.Hq + g * G + h) * kHeadDim + d] = float_to_half_bits(o / lh[h]);
-        }
+        grid_dep_launch();
+        cluster_wait();
+        cluster_arrive_release();
+        cluster_wait();
         return;
     }
 
-    // ---- split partials and the last-arriving merge
-    const size_t cell0 = (((size_t)b * p.Hkv + g) * p.splits) * G;  // (b, g, split 0, head 0)
+    // ---------------- consumers
+    grid_dep_wait();  // q comes from the preceding kernel
+    grid_dep_launch();
+    const int gq = lane >> 2, tig = lane & 3;  // MMA group (row) and thread-in-group
+    uint32_t qa[8][2];
+    {
+        const uint32_t *qrow = reinterpret_cast<const uint32_t *>(p.q + ((size_t)b * p.Hq + g * G + gq) * kHeadDim);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            qa[kk][0] = gq < G ? qrow[8 * kk + tig] : 0u;
+            qa[kk][1] = gq < G ? qrow[8 * kk + 4 + tig] : 0u;
+        }
+    }
+    const float qscale = p.scale * kLog2e;
+    float o[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    const int r8 = lane & 7, mi = lane >> 3;  // ldmatrix: row within an 8x8 matrix, matrix index
+    bool ok = true;
+    for (int i = 0; i < n_my; ++i) {
+        const int st = i % kStages, use = i / kStages;
+        if (ok && !mbar_wait(&full[st], (unsigned)(use & 1))) {
+            record_error(&g_attn_error, 1);
+            ok = false;
+        }
+        ok = __all_sync(0xffffffffu, ok);  // the MMAs and shuffles below need the whole warp
+        const int valid = ctx - ((tile0 + i) * kTileTokens + warp * kWarpTokens);  // tokens of this warp's 16
+        if (ok && valid > 0) {
+            const uint32_t kb = base + st * kStageBytes, vb = kb + 2 * kHalfBytes;
+            const int row0 = warp * kWarpTokens + r8;  // this lane's ldmatrix row for tokens 0-7 of the warp
+            // S[h][t] = q_h . k_t over 8 k-steps of 16 dims; s0: tokens 0-7, s1: tokens 8-15
+            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) {
+                const int chunk = 4 * k2 + mi;  // 16-byte chunk of the 256-byte row
+                const uint32_t off = (chunk >> 3) * kHalfBytes + (((chunk & 7) ^ r8) << 4);
+                uint32_t b0, b1, b2, b3, e0, e1, e2, e3;
+                ldsm_x4(kb + off + row0 * 128, b0, b1, b2, b3);
+                ldsm_x4(kb + off + (row0 + 8) * 128, e0, e1, e2, e3);
+                mma16816(s0, qa[2 * k2][0], 0u, qa[2 * k2][1], 0u, b0, b1);
+                mma16816(s1, qa[2 * k2][0], 0u, qa[2 * k2][1], 0u, e0, e1);
+                mma16816(s0, qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u, b2, b3);
+                mma16816(s1, qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u, e2, e3);
+            }
+            // this lane: head gq, tokens j, j+1, j+8, j+9 of the warp's 16
+            const int j = 2 * tig;
+            float sv[4] = {s0[0] * qscale, s0[1] * qscale, s1[0] * qscale, s1[1] * qscale};
+            uint32_t mk01 = 0xffffffffu, mk89 = 0xffffffffu;
+            if (valid < kWarpTokens) {
+                sv[0] = j < valid ? sv[0] : -INFINITY;
+                sv[1] = j + 1 < valid ? sv[1] : -INFINITY;
+                sv[2] = j + 8 < valid ? sv[2] : -INFINITY;
+                sv[3] = j + 9 < valid ? sv[3] : -INFINITY;
+                mk01 = (j < valid ? 0x0000ffffu : 0u) | (j + 1 < valid ? 0xffff0000u : 0u);
+                mk89 = (j + 8 < valid ? 0x0000ffffu : 0u) | (j + 9 < valid ? 0xffff0000u : 0u);
+            }
+            float mc = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+            mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, 1));
+            mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, 2));
+            const float m_new = fmaxf(m_run, mc);
+            const float m_use = m_new == -INFINITY ? 0.f : m_new;
+            const float alpha = exp2f(m_run - m_use);
+            const __half2 p01 = __floats2half2_rn(exp2f(sv[0] - m_use), exp2f(sv[1] - m_use));
+            const __half2 p89 = __floats2half2_rn(exp2f(sv[2] - m_use), exp2f(sv[3] - m_use));
+            const float2 f01 = __half22float2(p01), f89 = __half22float2(p89);
+            l_run = fmaf(l_run, alpha, (f01.x + f01.y) + (f89.x + f89.y));
+            m_run = m_new;
+            // O^T columns of this lane are heads 2*tig and 2*tig+1, whose rescale factors live in lanes 8*tig and 8*tig+4
+            const float a_lo = __shfl_sync(0xffffffffu, alpha, 8 * tig);
+            const float a_hi = __shfl_sync(0xffffffffu, alpha, 8 * tig + 4);
+            const uint32_t pb0 = h2_bits(p01), pb1 = h2_bits(p89);
+#pragma unroll
+            for (int im = 0; im < 8; ++im) {
+                // V^T tile: dims 16*im.., tokens 0-15 of the warp; matrices (t0-7, d lo), (t0-7, d hi), (t8-15, d lo), (t8-15, d hi)
+                const int chunk = 2 * im + (mi & 1);
+                const int row = warp * kWarpTokens + (mi >> 1) * 8 + r8;
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_trans(vb + (chunk >> 3) * kHalfBytes + row * 128 + (((chunk & 7) ^ r8) << 4), a0, a1, a2, a3);
+                o[im][0] *= a_lo;
+                o[im][1] *= a_hi;
+                o[im][2] *= a_lo;
+                o[im][3] *= a_hi;
+                mma16816(o[im], a0 & mk01, a1 & mk01, a2 & mk89, a3 & mk89, pb0, pb1);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+
+    // ---------------- merge the 4 warps (ring stage 0 becomes the partial buffer)
+    const int d = tid;  // the output dim this thread merges
+    float *wo = reinterpret_cast<float *>(gbase);  // [warp][dim][head]
+    consumer_sync();
+    if (tig == 0) wml[warp][gq] = make_float2(m_run, l_run);
+#pragma unroll
+    for (int im = 0; im < 8; ++im) {
+        float *r = wo + ((size_t)warp * kHeadDim + 16 * im + gq) * kMaxGroup + 2 * tig;
+        *reinterpret_cast<float2 *>(r) = make_float2(o[im][0], o[im][1]);
+        *reinterpret_cast<float2 *>(r + 8 * kMaxGroup) = make_float2(o[im][2], o[im][3]);
+    }
+    consumer_sync();
+    if (tid < kMaxGroup) {
+        const int h = tid;
+        float M = -INFINITY;
+        for (int k = 0; k < kConsumerWarps; ++k) M = fmaxf(M, wml[k][h].x);
+        float L = 0.f;
+        for (int k = 0; k < kConsumerWarps; ++k) {
+            const float wt = merge_weight(wml[k][h].x, M);
+            cw[k][h] = wt;
+            L = fmaf(wt, wml[k][h].y, L);
+        }
+        cM[h] = M;
+        cL[h] = L;
+    }
+    consumer_sync();
+    float oh[kMaxGroup];
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) oh[h] = 0.f;
+#pragma unroll
+    for (int k = 0; k < kConsumerWarps; ++k) {
+        const float4 lo = *reinterpret_cast<const float4 *>(wo + ((size_t)k * kHeadDim + d) * kMaxGroup);
+        const float4 hi = *reinterpret_cast<const float4 *>(wo + ((size_t)k * kHeadDim + d) * kMaxGroup + 4);
+        oh[0] = fmaf(cw[k][0], lo.x, oh[0]);
+        oh[1] = fmaf(cw[k][1], lo.y, oh[1]);
+        oh[2] = fmaf(cw[k][2], lo.z, oh[2]);
+        oh[3] = fmaf(cw[k][3], lo.w, oh[3]);
+        oh[4] = fmaf(cw[k][4], hi.x, oh[4]);
+        oh[5] = fmaf(cw[k][5], hi.y, oh[5]);
+        oh[6] = fmaf(cw[k][6], hi.z, oh[6]);
+        oh[7] = fmaf(cw[k][7], hi.w, oh[7]);
+    }
+
+    // ---------------- push this CTA's partial into the cluster leader (rank 0)
+    cluster_wait();  // every CTA of the cluster has started
+    {
+        const uint32_t dst = map_to_rank(base + kRecvOff + ((rank * kHeadDim + d) * kMaxGroup) * 4, 0);
+        st_cluster_f4(dst, oh[0], oh[1], oh[2], oh[3]);
+        st_cluster_f4(dst + 16, oh[4], oh[5], oh[6], oh[7]);
+        if (d < kMaxGroup) st_cluster_f2(map_to_rank(base + kRecvMlOff + (rank * kMaxGroup + d) * 8, 0), cM[d], cL[d]);
+    }
+    cluster_arrive_release();
+    cluster_wait();
+    if (rank != 0) return;
+
+    // ---------------- leader: merge the cluster's CTAs
+    const float *co = reinterpret_cast<const float *>(gbase + kRecvOff);
+    const float2 *cml = reinterpret_cast<const float2 *>(gbase + kRecvMlOff);
+    if (tid < kMaxGroup) {
+        const int h = tid;
+        float M = -INFINITY;
+        for (int k = 0; k < CL; ++k) M = fmaxf(M, cml[k * kMaxGroup + h].x);
+        float L = 0.f;
+        for (int k = 0; k < CL; ++k) {
+            const float wt = merge_weight(cml[k * kMaxGroup + h].x, M);
+            cw[k][h] = wt;
+            L = fmaf(wt, cml[k * kMaxGroup + h].y, L);
+        }
+        cM[h] = M;
+        cL[h] = L;
+    }
+    consumer_sync();
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) oh[h] = 0.f;
+    for (int k = 0; k < CL; ++k) {
+        const float4 lo = *reinterpret_cast<const float4 *>(co + ((size_t)k * kHeadDim + d) * kMaxGroup);
+        const float4 hi = *reinterpret_cast<const float4 *>(co + ((size_t)k * kHeadDim + d) * kMaxGroup + 4);
+        oh[0] = fmaf(cw[k][0], lo.x, oh[0]);
+        oh[1] = fmaf(cw[k][1], lo.y, oh[1]);
+        oh[2] = fmaf(cw[k][2], lo.z, oh[2]);
+        oh[3] = fmaf(cw[k][3], lo.w, oh[3]);
+        oh[4] = fmaf(cw[k][4], hi.x, oh[4]);
+        oh[5] = fmaf(cw[k][5], hi.y, oh[5]);
+        oh[6] = fmaf(cw[k][6], hi.z, oh[6]);
+        oh[7] = fmaf(cw[k][7], hi.w, oh[7]);
+    }
+    uint16_t *out = p.out + ((size_t)b * p.Hq + g * G) * kHeadDim + d;
+    if (w.clusters == 1) {
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+            if (h < G) out[(size_t)h * kHeadDim] = float_to_half_bits(oh[h] / cL[h]);
+        return;
+    }
+
+    // ---------------- several clusters: partials through the workspace, the last leader merges
+    const int cid = s / CL, n_cl = w.clusters;
+    const int max_cl = p.splits / CL;
+    const size_t cell0 = ((size_t)b * p.Hkv + g) * max_cl * G;  // (b, g, cluster 0, head 0)
     float2 *ml = reinterpret_cast<float2 *>(p.ws + p.ml_off);
     float *pacc = reinterpret_cast<float *>(p.ws + p.acc_off);
     unsigned *counter = reinterpret_cast<unsigned *>(p.ws + p.counters_off) + (size_t)b * p.Hkv + g;
-    for (int i = tid; i < G * kHeadDim; i += kAttnThreads) {
-        const int h = i / kHeadDim, d = i % kHeadDim;
-        const float o = (red[0][h][d] + red[1][h][d]) + (red[2][h][d] + red[3][h][d]);
-        pacc[(cell0 + (size_t)s * G + h) * kHeadDim + d] = o;
-    }
-    if (tid < G) ml[cell0 + (size_t)s * G + tid] = make_float2(mh[tid], lh[tid]);
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h)
+        if (h < G) pacc[(cell0 + (size_t)cid * G + h) * kHeadDim + d] = oh[h];
+    if (d < G) ml[cell0 + (size_t)cid * G + d] = make_float2(cM[d], cL[d]);
     __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const unsigned prev = atomicAdd(counter, 1u);
-        is_last = (prev == (unsigned)active - 1u);
-    }
-    __syncthreads();
+    consumer_sync();
+    if (tid == 0) is_last = atomicAdd(counter, 1u) == (unsigned)n_cl - 1u;
+    consumer_sync();
     if (!is_last) return;
     __threadfence();
-
-    // every split's (m, l) into shared memory at once (one coalesced pass), then per head
-    // (warp w takes heads w, w + 4) the maximum and the normalised weights 2^(m_j - M) / L
-    for (int i = tid; i < active * G; i += kAttnThreads) {
+    float *coef = reinterpret_cast<float *>(gbase + kRecvOff);  // [kMaxGroup][kMaxSplits]
+    float *lsum = coef + kMaxGroup * kMaxSplits;
+    for (int i = tid; i < n_cl * G; i += kConsumerThreads) {
         const float2 v = __ldcg(&ml[cell0 + i]);
-        coef[i % G][i / G] = v.x;
-        lsum[i % G][i / G] = v.y;
+        coef[(i % G) * kMaxSplits + i / G] = v.x;
+        lsum[(i % G) * kMaxSplits + i / G] = v.y;
     }
-    __syncthreads();
-    {
-        const int warp = tid >> 5, lane = tid & 31;
-        for (int h = warp; h < G; h += 4) {
-            float M = -INFINITY;
-            for (int j = lane; j < active; j += 32) M = fmaxf(M, coef[h][j]);
+    consumer_sync();
+    for (int h = warp; h < G; h += kConsumerWarps) {  // warp w: heads w, w+4
+        float *ch = coef + h * kMaxSplits;
+        const float *lh = lsum + h * kMaxSplits;
+        float M = -INFINITY;
+        for (int k = lane; k < n_cl; k += 32) M = fmaxf(M, ch[k]);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-            float L = 0.f;
-            for (int j = lane; j < active; j += 32) {
-                const float w = exp2f(coef[h][j] - M);
-                coef[h][j] = w;
-                L = fmaf(w, lsum[h][j], L);
-            }
-            L = warp_sum(L);
-            const float invL = 1.0f / L;
-            __syncwarp();
-            for (int j = lane; j < active; j += 32) coef[h][j] *= invL;
+        for (int sh = 16; sh > 0; sh >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
+        float L = 0.f;
+        for (int k = lane; k < n_cl; k += 32) {
+            const float wt = merge_weight(ch[k], M);
+            ch[k] = wt;
+            L = fmaf(wt, lh[k], L);
         }
+        L = warp_sum(L);
+        const float inv = 1.0f / L;
+        __syncwarp();
+        for (int k = lane; k < n_cl; k += 32) ch[k] *= inv;
     }
-    __syncthreads();
-    for (int i = tid; i < G * kHeadDim; i += kAttnThreads) {
-        const int h = i / kHeadDim, d = i % kHeadDim;
-        float o = 0.f;
-#pragma unroll 16
-        for (int j = 0; j < active; ++j) o = fmaf(coef[h][j], __ldcg(&pacc[(cell0 + (size_t)j * G + h) * kHeadDim + d]), o);
-        p.out[((size_t)b * p.Hq + g * G + h) * kHeadDim + d] = float_to_half_bits(o);
+    consumer_sync();
+    // four clusters' partials of every head per pass, all loads issued before the first use
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) oh[h] = 0.f;
+    for (int k0 = 0; k0 < n_cl; k0 += 4) {
+        float v[kMaxGroup][4];
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                v[h][u] = (h < G && k0 + u < n_cl) ? __ldcg(&pacc[(cell0 + (size_t)(k0 + u) * G + h) * kHeadDim + d])
+                                                   : 0.f;
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (h < G && k0 + u < n_cl) oh[h] = fmaf(coef[h * kMaxSplits + k0 + u], v[h][u], oh[h]);
     }
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h)
+        if (h < G) out[(size_t)h * kHeadDim] = float_to_half_bits(oh[h]);
     if (tid == 0) *counter = 0u;  // ready for the next call
 }
 
-int launch_paged_gqa_decode(const AttnParams &p_in, cudaStream_t stream, bool pdl) {
-    AttnParams p = p_in;
-    p.tile_tokens = attn_tile_tokens(p);
-    const int smem = 2 * p.tile_tokens * kHeadDim * 2;
-    static int configured = -1;
-    if (smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(paged_gqa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return cuda_check(e, "paged_gqa_decode smem attribute");
-        configured = smem;
-    }
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static int encoder(EncodeTiledFn *out) {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    static cudaError_t err = cudaSuccess;
+    static cudaDriverEntryPointQueryResult found = cudaDriverEntryPointSymbolNotFound;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        err = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &found);
+        fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    if (err != cudaSuccess) return cuda_check(err, "looking up cuTensorMapEncodeTiled");
+    if (found != cudaDriverEntryPointSuccess || !fn) return fail(I4_ECUDA, "cuTensorMapEncodeTiled not found in the driver");
+    *out = fn;
+    return I4_OK;
+}
+
+// [rows][128] fp16 view of a KV pool ([pages][Hkv][P][128]); box 64 dims x min(P, 64) rows, 128-byte swizzle
+static int encode_pool_map(CUtensorMap *map, const uint16_t *pool, int page_size) {
+    EncodeTiledFn fn = nullptr;
+    int st = encoder(&fn);
+    if (st) return st;
+    const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)kPoolRows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)(page_size < kTileTokens ? page_size : kTileTokens)};
+    const cuuint32_t estride[2] = {1u, 1u};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t *>(pool), dims, strides, box,
+                          estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(I4_ECUDA, "paged_gqa_decode: tensor map encoding failed (CUresult %d)", (int)r);
+    return I4_OK;
+}
+
+int launch_paged_gqa_decode(const AttnParams &p, cudaStream_t stream, bool pdl) {
+    AttnMaps maps;
+    int st = encode_pool_map(&maps.k, p.k_pool, p.page_size);
+    if (st) return st;
+    if ((st = encode_pool_map(&maps.v, p.v_pool, p.page_size))) return st;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(paged_gqa_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
+    });
+    if (attr_err != cudaSuccess) return cuda_check(attr_err, "paged_gqa_decode smem attribute");
     if (g_dry_run) return I4_OK;
-    return cuda_check(launch(paged_gqa_decode_kernel, dim3(p.splits, p.Hkv, p.B), dim3(kAttnThreads), (size_t)smem,
-                             stream, pdl, p),
-                      "paged_gqa_decode launch");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.splits, p.Hkv, p.B);
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = kDynSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    return cuda_check(cudaLaunchKernelEx(&cfg, paged_gqa_decode_kernel, maps, p), "paged_gqa_decode launch");
 }
 
 int read_attn_error(int reset) {
@@ -375,9 +609,9 @@ static int attn_check(const uint16_t *q, const uint16_t *k_pool, const uint16_t 
     if (B < 1 || Hq < 1 || Hkv < 1 || max_pages < 1) return fail(I4_EINVAL, "paged_gqa_decode: bad sizes");
     if (D != 128) return fail(I4_EUNSUPPORTED, "paged_gqa_decode: head_dim %d (only 128)", D);
     if (Hq % Hkv != 0 || Hq / Hkv > 8) return fail(I4_EUNSUPPORTED, "paged_gqa_decode: Hq/Hkv must be an integer <= 8");
-    if (page_size < 8 || page_size > kMaxTokensPerSplit || (page_size & (page_size - 1)))
+    if (page_size < 8 || page_size > kMaxPageSize || (page_size & (page_size - 1)))
         return fail(I4_EUNSUPPORTED, "paged_gqa_decode: page_size %d must be a power of two in [8, %d]", page_size,
-                    kMaxTokensPerSplit);
+                    kMaxPageSize);
     if (B > 65535 || Hkv > 65535) return fail(I4_EUNSUPPORTED, "paged_gqa_decode: grid too large");
     if ((long long)max_pages * page_size > kMaxCtx)
         return fail(I4_EUNSUPPORTED, "paged_gqa_decode: max_pages_per_seq * page_size above %d tokens", kMaxCtx);
@@ -416,6 +650,7 @@ extern "C" int paged_gqa_decode(const uint16_t *q, const uint16_t *k_pool, const
     p.max_pages = max_pages_per_seq;
     p.scale = scale;
     p.splits = L.splits;
+    p.cluster = L.cluster;
     p.ws = reinterpret_cast<char *>(ws);
     p.counters_off = L.counters_off;
     p.ml_off = L.ml_off;
@@ -486,6 +721,7 @@ extern "C" int paged_gqa_decode_static(const uint16_t *q, const uint16_t *k_pool
     p.max_pages = max_pages_per_seq;
     p.scale = scale;
     p.splits = L.splits;
+    p.cluster = L.cluster;
     p.ws = ws;
     p.counters_off = L.counters_off;
     p.ml_off = L.ml_off;

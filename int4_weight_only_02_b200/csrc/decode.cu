@@ -108,6 +108,7 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
             p.page_size = d.page_size;
             p.max_pages = max_pages;
             p.splits = g->attn_layout.splits;
+            p.cluster = g->attn_layout.cluster;
             p.scale = (float)(1.0 / std::sqrt((double)D));
             p.ws = g->attn_ws;
             p.counters_off = g->attn_layout.counters_off;

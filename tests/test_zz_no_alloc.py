@@ -43,7 +43,7 @@ def test_static_scratch_matches_workspace_variant_on_consecutive_calls(i4lib, cu
 
 def test_static_scratch_refuses_oversized_shapes(i4lib):
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check comes first
-    # 64 sequences x 8 kv heads at 32k context need far more than the fixed scratch
-    st = i4lib.lib().paged_gqa_decode_static(fake, fake, fake, fake, fake, fake, 64, 64, 8, 128, 64, 512, 1.0, None)
+    # 4096 sequences x 8 kv heads need 4 KB of fp32 partials per head, far more than the fixed scratch
+    st = i4lib.lib().paged_gqa_decode_static(fake, fake, fake, fake, fake, fake, 4096, 64, 8, 128, 64, 512, 1.0, None)
     assert st == i4lib.I4_EUNSUPPORTED
     assert b"static scratch" in i4lib.lib().i4_last_error()
