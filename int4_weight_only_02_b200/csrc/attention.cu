@@ -12,14 +12,16 @@
 //  * Work. Grid (S, Hkv, B) in clusters of CL CTAs along x. The context of
 //    sequence b is cut into tiles of 64 tokens and CTA s takes tiles
 //    [s*tpc, (s+1)*tpc). tpc comes from ctx_len[b] on the device, so a captured
-//    graph stays valid as the context grows; contexts of up to 2*CL tiles stay
+//    graph stays valid as the context grows; contexts of up to 8*CL tiles stay
 //    inside one cluster.
-//  * Data. A producer warp brings each tile's K and V rows into a two-stage
-//    shared-memory ring with 2-D TMA copies (one per page piece and 64-dim
-//    half, 128-byte swizzle, no multicast). A page below the one holding
-//    position ctx-1 was written by an earlier step, so its copy is issued before
-//    the programmatic dependency wait; the current page after it.
-//  * Math. Each of 4 consumer warps takes 16 tokens of a tile.
+//  * Data. Every warp stages its own 16 tokens of each tile: 16-byte cp.async
+//    copies from the pool pages into a per-warp two-stage shared-memory ring,
+//    each 64-dim half of a row at 128 bytes with its 16-byte chunks XOR-swizzled
+//    by row, so the ldmatrix reads below are free of bank conflicts. Page-table
+//    entries are read 32 tiles ahead. A page below the one holding position
+//    ctx-1 was written by an earlier step, so its copies are issued before the
+//    programmatic dependency wait; the current page's after it.
+//  * Math. Each of the 4 warps takes 16 tokens of a tile.
 //    S = Q K^T on mma.m16n8k16 with the G <= 8 query heads that share the kv
 //    head as the M rows (rows G..15 are zero), so each K row is read once for
 //    all G heads. P = 2^(S - m) rounded to fp16 then feeds O^T = V^T P^T
@@ -31,8 +33,6 @@
 //    output; otherwise cluster leaders write partials to the workspace and the
 //    last to arrive merges them:
 //      M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
-#include <cuda.h>  // CUtensorMap and its enums; the encoder is looked up in the driver at run time
-
 #include <mutex>
 
 #include "async.cuh"
@@ -42,33 +42,32 @@
 namespace i4 {
 
 constexpr int kHeadDim = 128;
-constexpr int kMaxGroup = 8;                               // query heads per kv head (MMA rows used)
-constexpr int kWarpTokens = 16;                            // tokens of a tile per consumer warp
-constexpr int kConsumerWarps = 4;
-constexpr int kTileTokens = kConsumerWarps * kWarpTokens;  // 64
-constexpr int kStages = 2;
-constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kAttnThreads = kConsumerThreads + 32;        // + the producer warp
+constexpr int kMaxGroup = 8;                        // query heads per kv head (MMA rows used)
+constexpr int kWarpTokens = 16;                     // tokens of a tile per warp
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTileTokens = kWarps * kWarpTokens;   // 64
+constexpr int kStages = 2;                          // ring depth of every warp
 constexpr int kMaxCluster = 8;
-constexpr int kOneClusterTiles = 2;  // contexts up to kMaxCluster * this many tiles stay in one cluster
+constexpr int kOneClusterTiles = 8;  // contexts up to kMaxCluster * this many tiles stay in one cluster
 constexpr int kMaxSplits = 256;
 constexpr int kMaxCtx = 32768;
 constexpr int kMaxPageSize = 128;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr unsigned long long kPoolRows = (1ull << 31) - 1;  // row bound of the pool tensor maps (rows are int32)
 
-// Dynamic shared memory, from a 1024-byte aligned base (128-byte swizzle atoms):
-//   ring  kStages x {K dims 0-63, K dims 64-127, V dims 0-63, V dims 64-127}, each [64 tokens][128 B]
+// Dynamic shared memory (128-byte aligned base):
+//   ring  [warp][stage] {K dims 0-63, K dims 64-127, V dims 0-63, V dims 64-127}, each [16 tokens][128 B]
 //   recv  [kMaxCluster][kHeadDim][kMaxGroup] fp32 o and [kMaxCluster][kMaxGroup] (m, l) pushed by the cluster
-// The warp partials reuse ring stage 0 once every tile is consumed; the cross-cluster merge reuses recv.
-constexpr unsigned kHalfBytes = kTileTokens * 128;
-constexpr unsigned kStageBytes = 4 * kHalfBytes;
-constexpr unsigned kRingBytes = kStages * kStageBytes;
+// The warp partials reuse the ring once every tile is consumed; the cross-cluster merge reuses recv.
+constexpr unsigned kRegionBytes = kWarpTokens * 128;
+constexpr unsigned kWarpStageBytes = 4 * kRegionBytes;
+constexpr unsigned kRingBytes = kWarps * kStages * kWarpStageBytes;
 constexpr unsigned kRecvOff = kRingBytes;
 constexpr unsigned kRecvBytes = kMaxCluster * kHeadDim * kMaxGroup * 4;
 constexpr unsigned kRecvMlOff = kRecvOff + kRecvBytes;
-constexpr unsigned kDynSmem = 1024 + kRecvMlOff + kMaxCluster * kMaxGroup * 8;
-static_assert(kConsumerWarps * kHeadDim * kMaxGroup * 4 <= kStageBytes, "warp partials must fit in one stage");
+constexpr unsigned kDynSmem = 128 + kRecvMlOff + kMaxCluster * kMaxGroup * 8;
+constexpr int kCtasPerSm = (228 * 1024) / (kDynSmem + 2048);  // with the static part and the per-CTA reserve
+static_assert(kWarps * kHeadDim * kMaxGroup * 4 <= kRingBytes, "warp partials must fit in the ring");
 static_assert(2 * kMaxGroup * kMaxSplits * 4 <= kRecvBytes, "merge weights must fit in the receive buffer");
 
 __device__ int g_attn_error = 0;
@@ -89,10 +88,10 @@ __host__ __device__ inline Split split_work(int n_tiles, int splits, int cl) {
 }
 
 AttnWs attn_ws_layout(int B, int Hq, int Hkv, int page_size, int max_pages) {
-    // about two CTAs per SM over the grid, whole clusters, no more CTAs than tiles
+    // one wave of CTAs over the SMs, whole clusters, no more CTAs than tiles
     const int max_tiles = (int)(((long long)max_pages * page_size + kTileTokens - 1) / kTileTokens);
     const int rows = B * Hkv;
-    int s = (2 * kNumSMs + rows - 1) / rows;
+    int s = (kCtasPerSm * kNumSMs + rows - 1) / rows;
     s = s < max_tiles ? s : max_tiles;
     s = s < kMaxSplits ? s : kMaxSplits;
     s = s < 1 ? 1 : s;
@@ -111,17 +110,12 @@ AttnWs attn_ws_layout(int B, int Hq, int Hkv, int page_size, int max_pages) {
 
 // ------------------------------------------------------------------ device helpers
 
-struct __align__(64) AttnMaps {
-    CUtensorMap k, v;  // [rows = pages*Hkv*P][128] fp16 views of the pools, box 64 dims x min(P, 64) rows
-};
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-            "r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -164,7 +158,6 @@ __device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, f
 __device__ __forceinline__ void st_cluster_f2(uint32_t addr, float a, float b) {
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
 }
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory"); }
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 
 // weight of a partial with maximum m under the merged maximum M (0 for an empty partial)
@@ -174,10 +167,8 @@ __device__ __forceinline__ float merge_weight(float m, float M) {
 
 // ------------------------------------------------------------------ the kernel
 
-__global__ void __launch_bounds__(kAttnThreads, 2)
-    paged_gqa_decode_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) paged_gqa_decode_kernel(const AttnParams p) {
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
     __shared__ float2 wml[kMaxCluster][kMaxGroup];  // (m, l) of the 4 warps, later of the cluster's CTAs
     __shared__ float cw[kMaxCluster][kMaxGroup];    // merge weights
     __shared__ float cM[kMaxGroup], cL[kMaxGroup];
@@ -199,59 +190,70 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     n_my = n_my < 0 ? 0 : (n_my > w.tpc ? w.tpc : n_my);
 
     const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
+    const uint32_t base = (raw + 127u) & ~127u;
     unsigned char *gbase = smem_raw + (base - raw);
+    const uint32_t ring = base + warp * kStages * kWarpStageBytes;  // this warp's stages
 
-    if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kConsumerWarps);
+    // ---------------- staging: lane copies 16-byte chunk (lane & 15) of rows (lane >> 4) + 2j, j < 8
+    const int last_page = (ctx - 1) / P;
+    const int32_t *table = p.page_table + (size_t)b * p.max_pages;
+    const size_t head_rows = (size_t)g * P;  // row offset of kv head g inside a page
+    auto slab = [&](int i) { return (tile0 + i) * kTileTokens + warp * kWarpTokens; };  // first token of tile i
+    // page-table entries of the pages holding the first and the last token of the warp's 16, 32 tiles per batch
+    auto fetch = [&](int batch, int &ea, int &eb) {
+        const int i = batch * 32 + lane;
+        const int t = slab(i);
+        ea = eb = 0;
+        if (i < n_my && t < ctx) {
+            const int tl = t + kWarpTokens - 1 < ctx ? t + kWarpTokens - 1 : ctx - 1;
+            ea = table[t / P];
+            eb = table[tl / P];
         }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-
-    if (warp == kConsumerWarps) {
-        // ---------------- producer: lane = piece * 4 + part (K lo, K hi, V lo, V hi)
-        const int R = P < kTileTokens ? P : kTileTokens;  // rows per copy: one page, or 64 rows of a larger page
-        const int pieces = kTileTokens / R;
-        const int last_page = (ctx - 1) / P;
-        const int32_t *table = p.page_table + (size_t)b * p.max_pages;
-        bool waited = false;
-        for (int i = 0; i < n_my; ++i) {
-            const int st = i % kStages, use = i / kStages;
-            if (use > 0 && !mbar_wait(&empty[st], (unsigned)((use - 1) & 1))) {
-                record_error(&g_attn_error, 1);
-                break;
-            }
-            const int t0 = (tile0 + i) * kTileTokens;
-            int n_pc = (ctx - t0 + R - 1) / R;
-            n_pc = n_pc < pieces ? n_pc : pieces;
-            if (!waited && (t0 + n_pc * R - 1) / P >= last_page) {
+    };
+    int cur_batch = 0, ca, cb, na, nb;
+    fetch(0, ca, cb);
+    fetch(1, na, nb);
+    const int chunk = lane & 15, row_lo = lane >> 4;
+    const uint32_t chunk_off = (chunk >> 3) * kRegionBytes;  // K: dims 0-63 or 64-127
+    bool waited = false;
+    auto issue = [&](int i) {  // tile i into stage i % kStages (warp-uniform control flow)
+        const int batch = i >> 5;
+        while (cur_batch < batch) {
+            ca = na;
+            cb = nb;
+            fetch(++cur_batch + 1, na, nb);
+        }
+        const int ea = __shfl_sync(0xffffffffu, ca, i & 31), eb = __shfl_sync(0xffffffffu, cb, i & 31);
+        const int t = slab(i);
+        if (!waited && t < ctx) {
+            const int tl = t + kWarpTokens - 1 < ctx ? t + kWarpTokens - 1 : ctx - 1;
+            if (tl / P == last_page) {
                 grid_dep_wait();  // the current page's new row comes from the preceding kernel
-                asm volatile("fence.proxy.async;" ::: "memory");
                 waited = true;
             }
-            if (lane == 0) mbar_expect_tx(&full[st], (unsigned)(n_pc * 4 * R * 128));
-            __syncwarp();
-            if (lane < n_pc * 4) {
-                const int pc = lane >> 2, part = lane & 3;
-                const int t = t0 + pc * R;
-                const int y = (table[t / P] * p.Hkv + g) * P + (t % P);
-                const uint32_t dst = base + st * kStageBytes + part * kHalfBytes + pc * R * 128;
-                tma_load_2d(dst, part < 2 ? &maps.k : &maps.v, (part & 1) * 64, y, &full[st]);
+        }
+        const uint32_t st = ring + (i % kStages) * kWarpStageBytes + chunk_off;
+        const int pa = t / P;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int r = row_lo + 2 * j, tok = t + r;
+            if (tok < ctx) {
+                const int e = tok / P == pa ? ea : eb;
+                const size_t row = ((size_t)e * p.Hkv) * P + head_rows + (tok % P);
+                const uint32_t dst = st + r * 128 + (((chunk & 7) ^ (r & 7)) << 4);
+                cp_async16(dst, p.k_pool + row * kHeadDim + chunk * 8);
+                cp_async16(dst + 2 * kRegionBytes, p.v_pool + row * kHeadDim + chunk * 8);
             }
         }
-        grid_dep_launch();
-        cluster_wait();
-        cluster_arrive_release();
-        cluster_wait();
-        return;
+    };
+#pragma unroll 1
+    for (int i = 0; i < kStages; ++i) {
+        if (i < n_my) issue(i);
+        cp_async_commit();
     }
-
-    // ---------------- consumers
-    grid_dep_wait();  // q comes from the preceding kernel
+    if (!waited) grid_dep_wait();  // q comes from the preceding kernel
     grid_dep_launch();
+
     const int gq = lane >> 2, tig = lane & 3;  // MMA group (row) and thread-in-group
     uint32_t qa[8][2];
     {
@@ -268,27 +270,22 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m_run = -INFINITY, l_run = 0.f;
     const int r8 = lane & 7, mi = lane >> 3;  // ldmatrix: row within an 8x8 matrix, matrix index
-    bool ok = true;
+#pragma unroll 1
     for (int i = 0; i < n_my; ++i) {
-        const int st = i % kStages, use = i / kStages;
-        if (ok && !mbar_wait(&full[st], (unsigned)(use & 1))) {
-            record_error(&g_attn_error, 1);
-            ok = false;
-        }
-        ok = __all_sync(0xffffffffu, ok);  // the MMAs and shuffles below need the whole warp
-        const int valid = ctx - ((tile0 + i) * kTileTokens + warp * kWarpTokens);  // tokens of this warp's 16
-        if (ok && valid > 0) {
-            const uint32_t kb = base + st * kStageBytes, vb = kb + 2 * kHalfBytes;
-            const int row0 = warp * kWarpTokens + r8;  // this lane's ldmatrix row for tokens 0-7 of the warp
+        cp_async_wait<kStages - 1>();  // this lane's copies of tile i have landed
+        __syncwarp();                  // and every other lane's
+        const int valid = ctx - slab(i);  // tokens of this warp's 16 that exist
+        if (valid > 0) {
+            const uint32_t kb = ring + (i % kStages) * kWarpStageBytes, vb = kb + 2 * kRegionBytes;
             // S[h][t] = q_h . k_t over 8 k-steps of 16 dims; s0: tokens 0-7, s1: tokens 8-15
             float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int k2 = 0; k2 < 4; ++k2) {
-                const int chunk = 4 * k2 + mi;  // 16-byte chunk of the 256-byte row
-                const uint32_t off = (chunk >> 3) * kHalfBytes + (((chunk & 7) ^ r8) << 4);
+                const int c = 4 * k2 + mi;  // 16-byte chunk of the 256-byte row
+                const uint32_t off = (c >> 3) * kRegionBytes + (((c & 7) ^ r8) << 4);
                 uint32_t b0, b1, b2, b3, e0, e1, e2, e3;
-                ldsm_x4(kb + off + row0 * 128, b0, b1, b2, b3);
-                ldsm_x4(kb + off + (row0 + 8) * 128, e0, e1, e2, e3);
+                ldsm_x4(kb + off + r8 * 128, b0, b1, b2, b3);
+                ldsm_x4(kb + off + (r8 + 8) * 128, e0, e1, e2, e3);
                 mma16816(s0, qa[2 * k2][0], 0u, qa[2 * k2][1], 0u, b0, b1);
                 mma16816(s1, qa[2 * k2][0], 0u, qa[2 * k2][1], 0u, e0, e1);
                 mma16816(s0, qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u, b2, b3);
@@ -323,11 +320,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             const uint32_t pb0 = h2_bits(p01), pb1 = h2_bits(p89);
 #pragma unroll
             for (int im = 0; im < 8; ++im) {
-                // V^T tile: dims 16*im.., tokens 0-15 of the warp; matrices (t0-7, d lo), (t0-7, d hi), (t8-15, d lo), (t8-15, d hi)
-                const int chunk = 2 * im + (mi & 1);
-                const int row = warp * kWarpTokens + (mi >> 1) * 8 + r8;
+                // V^T tile: dims 16*im.., the warp's 16 tokens; matrices (t0-7, d lo), (t0-7, d hi), (t8-15, d lo), (t8-15, d hi)
+                const int c = 2 * im + (mi & 1);
+                const int row = (mi >> 1) * 8 + r8;
                 uint32_t a0, a1, a2, a3;
-                ldsm_x4_trans(vb + (chunk >> 3) * kHalfBytes + row * 128 + (((chunk & 7) ^ r8) << 4), a0, a1, a2, a3);
+                ldsm_x4_trans(vb + (c >> 3) * kRegionBytes + row * 128 + (((c & 7) ^ r8) << 4), a0, a1, a2, a3);
                 o[im][0] *= a_lo;
                 o[im][1] *= a_hi;
                 o[im][2] *= a_lo;
@@ -335,16 +332,18 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                 mma16816(o[im], a0 & mk01, a1 & mk01, a2 & mk89, a3 & mk89, pb0, pb1);
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+        __syncwarp();  // every lane is done with this stage before it is refilled
+        if (i + kStages < n_my) issue(i + kStages);
+        cp_async_commit();
     }
+    cp_async_wait<0>();
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
 
-    // ---------------- merge the 4 warps (ring stage 0 becomes the partial buffer)
+    // ---------------- merge the 4 warps (the ring becomes the partial buffer)
     const int d = tid;  // the output dim this thread merges
     float *wo = reinterpret_cast<float *>(gbase);  // [warp][dim][head]
-    consumer_sync();
+    __syncthreads();
     if (tig == 0) wml[warp][gq] = make_float2(m_run, l_run);
 #pragma unroll
     for (int im = 0; im < 8; ++im) {
@@ -352,13 +351,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         *reinterpret_cast<float2 *>(r) = make_float2(o[im][0], o[im][1]);
         *reinterpret_cast<float2 *>(r + 8 * kMaxGroup) = make_float2(o[im][2], o[im][3]);
     }
-    consumer_sync();
+    __syncthreads();
     if (tid < kMaxGroup) {
         const int h = tid;
         float M = -INFINITY;
-        for (int k = 0; k < kConsumerWarps; ++k) M = fmaxf(M, wml[k][h].x);
+        for (int k = 0; k < kWarps; ++k) M = fmaxf(M, wml[k][h].x);
         float L = 0.f;
-        for (int k = 0; k < kConsumerWarps; ++k) {
+        for (int k = 0; k < kWarps; ++k) {
             const float wt = merge_weight(wml[k][h].x, M);
             cw[k][h] = wt;
             L = fmaf(wt, wml[k][h].y, L);
@@ -366,12 +365,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         cM[h] = M;
         cL[h] = L;
     }
-    consumer_sync();
+    __syncthreads();
     float oh[kMaxGroup];
 #pragma unroll
     for (int h = 0; h < kMaxGroup; ++h) oh[h] = 0.f;
 #pragma unroll
-    for (int k = 0; k < kConsumerWarps; ++k) {
+    for (int k = 0; k < kWarps; ++k) {
         const float4 lo = *reinterpret_cast<const float4 *>(wo + ((size_t)k * kHeadDim + d) * kMaxGroup);
         const float4 hi = *reinterpret_cast<const float4 *>(wo + ((size_t)k * kHeadDim + d) * kMaxGroup + 4);
         oh[0] = fmaf(cw[k][0], lo.x, oh[0]);
@@ -412,7 +411,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         cM[h] = M;
         cL[h] = L;
     }
-    consumer_sync();
+    __syncthreads();
 #pragma unroll
     for (int h = 0; h < kMaxGroup; ++h) oh[h] = 0.f;
     for (int k = 0; k < CL; ++k) {
@@ -447,20 +446,20 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         if (h < G) pacc[(cell0 + (size_t)cid * G + h) * kHeadDim + d] = oh[h];
     if (d < G) ml[cell0 + (size_t)cid * G + d] = make_float2(cM[d], cL[d]);
     __threadfence();
-    consumer_sync();
+    __syncthreads();
     if (tid == 0) is_last = atomicAdd(counter, 1u) == (unsigned)n_cl - 1u;
-    consumer_sync();
+    __syncthreads();
     if (!is_last) return;
     __threadfence();
     float *coef = reinterpret_cast<float *>(gbase + kRecvOff);  // [kMaxGroup][kMaxSplits]
     float *lsum = coef + kMaxGroup * kMaxSplits;
-    for (int i = tid; i < n_cl * G; i += kConsumerThreads) {
+    for (int i = tid; i < n_cl * G; i += kThreads) {
         const float2 v = __ldcg(&ml[cell0 + i]);
         coef[(i % G) * kMaxSplits + i / G] = v.x;
         lsum[(i % G) * kMaxSplits + i / G] = v.y;
     }
-    consumer_sync();
-    for (int h = warp; h < G; h += kConsumerWarps) {  // warp w: heads w, w+4
+    __syncthreads();
+    for (int h = warp; h < G; h += kWarps) {  // warp w: heads w, w+4
         float *ch = coef + h * kMaxSplits;
         const float *lh = lsum + h * kMaxSplits;
         float M = -INFINITY;
@@ -478,7 +477,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         __syncwarp();
         for (int k = lane; k < n_cl; k += 32) ch[k] *= inv;
     }
-    consumer_sync();
+    __syncthreads();
     // four clusters' partials of every head per pass, all loads issued before the first use
 #pragma unroll
     for (int h = 0; h < kMaxGroup; ++h) oh[h] = 0.f;
@@ -504,47 +503,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 
 // ------------------------------------------------------------------ host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static int encoder(EncodeTiledFn *out) {
-    static std::once_flag once;
-    static EncodeTiledFn fn = nullptr;
-    static cudaError_t err = cudaSuccess;
-    static cudaDriverEntryPointQueryResult found = cudaDriverEntryPointSymbolNotFound;
-    std::call_once(once, [] {
-        void *f = nullptr;
-        err = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &found);
-        fn = reinterpret_cast<EncodeTiledFn>(f);
-    });
-    if (err != cudaSuccess) return cuda_check(err, "looking up cuTensorMapEncodeTiled");
-    if (found != cudaDriverEntryPointSuccess || !fn) return fail(I4_ECUDA, "cuTensorMapEncodeTiled not found in the driver");
-    *out = fn;
-    return I4_OK;
-}
-
-// [rows][128] fp16 view of a KV pool ([pages][Hkv][P][128]); box 64 dims x min(P, 64) rows, 128-byte swizzle
-static int encode_pool_map(CUtensorMap *map, const uint16_t *pool, int page_size) {
-    EncodeTiledFn fn = nullptr;
-    int st = encoder(&fn);
-    if (st) return st;
-    const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)kPoolRows};
-    const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-    const cuuint32_t box[2] = {64u, (cuuint32_t)(page_size < kTileTokens ? page_size : kTileTokens)};
-    const cuuint32_t estride[2] = {1u, 1u};
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t *>(pool), dims, strides, box,
-                          estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(I4_ECUDA, "paged_gqa_decode: tensor map encoding failed (CUresult %d)", (int)r);
-    return I4_OK;
-}
-
 int launch_paged_gqa_decode(const AttnParams &p, cudaStream_t stream, bool pdl) {
-    AttnMaps maps;
-    int st = encode_pool_map(&maps.k, p.k_pool, p.page_size);
-    if (st) return st;
-    if ((st = encode_pool_map(&maps.v, p.v_pool, p.page_size))) return st;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
@@ -554,7 +513,7 @@ int launch_paged_gqa_decode(const AttnParams &p, cudaStream_t stream, bool pdl) 
     if (g_dry_run) return I4_OK;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.splits, p.Hkv, p.B);
-    cfg.blockDim = dim3(kAttnThreads);
+    cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kDynSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -566,7 +525,7 @@ int launch_paged_gqa_decode(const AttnParams &p, cudaStream_t stream, bool pdl) 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    return cuda_check(cudaLaunchKernelEx(&cfg, paged_gqa_decode_kernel, maps, p), "paged_gqa_decode launch");
+    return cuda_check(cudaLaunchKernelEx(&cfg, paged_gqa_decode_kernel, p), "paged_gqa_decode launch");
 }
 
 int read_attn_error(int reset) {
