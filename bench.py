@@ -102,21 +102,30 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def traffic_from_profile(kernel_src: str):
-    """DRAM bytes per launch of the gate/up GEMV from the committed ncu summary, if it
-    was taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "gemv_gate_up_qwen7b.md")
+GEMV_SOURCES = ["gemv_stream.cu", "gemv_parts.cuh", "gemv.cuh", "common.cuh", "async.cuh"]
+
+
+def sources_hash(names) -> str:
+    """First 16 hex digits of the sha256 over the named kernel sources, in order."""
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "int4_weight_only_02_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(profile: str, names):
+    """DRAM bytes (read + write) per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
     try:
-        text = open(path).read()
+        text = open(os.path.join(ROOT, "profiles", profile)).read()
     except OSError:
         return None
-    src_hash = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
     vals = {}
     for line in text.splitlines():
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             vals[k.strip()] = v.strip().strip("`")
-    if vals.get("source_sha256_16") != src_hash:
+    if vals.get("source_sha256_16") != sources_hash(names):
         return None
     try:
         return float(vals["dram_bytes_per_full_launch"])
@@ -244,6 +253,89 @@ def run_profile_kernel(args):
     return 0
 
 
+def run_attention_sweep(args):
+    """Paged decode attention sweep (contexts 512-32768, page sizes 16 and 64, batches 1/8/32,
+    ragged lengths uniform in [L/2, L], pages drawn from one shuffled shared pool): KV bytes read
+    per second against the measured HBM peak, one JSON line per case. Each case is timed as a
+    CUDA graph of (L2 flush, attention) pairs minus a graph of the flushes alone, so every launch
+    starts L2-cold. K/V values come from a seeded device generator (timing only; parity is the
+    tests' job)."""
+    import numpy as np
+    import torch
+
+    import int4_weight_only_02_b200 as i4
+    from int4_weight_only_02_b200 import synth
+    dev = torch.device("cuda", 0)
+    peak, peak_kind = measured_peaks()
+    gen = torch.Generator(device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    reps = 10
+
+    def graph_ms(body):
+        side = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(side):
+            body(side)  # warm-up outside the capture
+            with torch.cuda.graph(g, stream=side):
+                for _ in range(reps):
+                    body(side)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        best = None
+        for _ in range(3):
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) / reps
+            best = t if best is None else min(best, t)
+        return best
+
+    contexts = [int(c) for c in args.sweep_contexts.split(",")]
+    for L in contexts:
+        for P in (16, 64):
+            for B in (1, 8, 32):
+                lens = synth.ragged_lengths(L, B, seed=L + B) if B > 1 else np.array([L], np.int32)
+                need = [(int(n) + P - 1) // P for n in lens]
+                max_pages = max(need)
+                n_pool = sum(need)
+                perm = synth.rng_for(0, 7, L, P, B).permutation(n_pool).astype(np.int32)
+                table = np.zeros((B, max_pages), np.int32)
+                off = 0
+                for b, n in enumerate(need):
+                    table[b, :n] = perm[off:off + n]
+                    off += n
+                gen.manual_seed(L * 1000 + P * 10 + B)
+                kp = torch.randn((n_pool, 4, P, 128), generator=gen, device=dev).half()
+                vp = torch.randn((n_pool, 4, P, 128), generator=gen, device=dev).half()
+                q = torch.randn((B, 28, 128), generator=gen, device=dev).half()
+                tab = torch.from_numpy(table).to(dev)
+                ctx = torch.from_numpy(lens.astype(np.int32)).to(dev)
+                out = torch.empty_like(q)
+                ws = torch.zeros(i4.paged_gqa_decode_ws_bytes(B, 28, 4, 128, P, max_pages), dtype=torch.uint8,
+                                 device=dev)
+
+                def flush_only(st):
+                    flush.add_(1)
+
+                def both(st):
+                    flush.add_(1)
+                    i4.paged_gqa_decode(q, kp, vp, tab, ctx, out=out, ws=ws, stream=st)
+
+                ms = graph_ms(both) - graph_ms(flush_only)
+                kv = int(lens.astype(np.int64).sum()) * 4 * 128 * 2 * 2
+                gbs = kv / (ms * 1e-3) / 1e9
+                print(json.dumps({"sweep": "paged_gqa_decode", "ctx_max": L, "page_size": P, "batch": B,
+                                  "kv_bytes": kv, "us": round(ms * 1e3, 2), "GBs": round(gbs, 1),
+                                  "frac": round(gbs / peak, 4), "peak": peak, "peak_kind": peak_kind,
+                                  "device_error": i4.device_error()}), flush=True)
+                del kp, vp, q, out, ws
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -260,11 +352,16 @@ def main():
                          "decode step, --launches times (for ncu captures)")
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--prime-steps", type=int, default=0, help="profiling mode: decode steps run first")
+    ap.add_argument("--attention-sweep", action="store_true",
+                    help="paged attention sweep over contexts, page sizes 16/64 and batches 1/8/32 (KV GB/s)")
+    ap.add_argument("--sweep-contexts", default="512,2048,8192,32768")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.profile_kernel:
         return run_profile_kernel(args)
+    if args.attention_sweep:
+        return run_attention_sweep(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 
@@ -401,7 +498,7 @@ def main():
 
     peak, peak_kind = measured_peaks()
     gu_gbs = gu_bytes / (gu_ms * 1e-3) / 1e9
-    traffic = traffic_from_profile(os.path.join(ROOT, "int4_weight_only_02_b200", "csrc", "gemv.cu"))
+    traffic = traffic_from_profile("gemv_gate_up_qwen7b.md", GEMV_SOURCES)
 
     weight_bytes = model.weight_bytes()
     ctx_mean = (ctx0 + ctx1 - 1) / 2.0
