@@ -264,14 +264,16 @@ I4_API int decode_step_launch_kernel(i4_graph *g, int index, void *stream);
  *   "pdl"    0/1 (default 1): launch the kernels of a decode step with programmatic
  *            dependent launch (each kernel still waits for its predecessor's
  *            results before reading them);
- *   "unpack" 0..3: INT4 unpack / multiply variant of the GEMV: 0 exact fp16
+ *   "unpack" 0..4: INT4 unpack / multiply variant of the GEMV: 0 exact fp16
  *            values, 1 offset-binary fp16 subnormals with a sum(x) correction
  *            (both fp16 x fp16 -> fp32 FMAs), 2 fp32 values from an exponent
  *            trick (packed fp32 FMAs), 3 the subnormal fields as the A operand of
- *            mma.sync (tensor cores, fp32 accumulate);
+ *            mma.sync (tensor cores, fp32 accumulate), 4 (default) per launch: 3
+ *            for a single vector (M == 1), else 0;
  *   "stream" 0/1: use the bulk-copy pipelined GEMV where the shape allows it
  *            (M == 1, K % 512 == 0, 16-byte aligned w and scales), default 1;
- *   "stream_smem_kb" 32..227: shared memory budget of that kernel's ring.
+ *   "stream_smem_kb" 32..227: shared memory budget of that kernel's ring;
+ *   "gemv_ctas_per_sm" 1/2 (default 2): CTAs per SM of the pipelined GEMV grids.
  * Not thread-safe; set options before creating graphs.
  */
 I4_API int i4_set_option(const char *name, int value);
@@ -286,17 +288,10 @@ I4_API int i4_device_error(int reset);
 /*
  * int4_gemv with an explicit unpack variant (as for "unpack") and a cap on the
  * number of CTAs (0 = none; any cap selects the register-streaming kernel
- * instead of the bulk-copy pipelined one); for tests and benchmarks. With
- * unpack 3, K > 4096 and a workspace (ws != NULL, ws_bytes >=
- * i4_int4_gemv_ksplit_ws_bytes(N, K), 256-byte aligned, zeroed before first
- * use and left zeroed) the K-split tensor-core kernel runs; without one the
- * call falls back to unpack 1.
+ * instead of the bulk-copy pipelined one); for tests and benchmarks.
  */
 I4_API int i4_int4_gemv_variant(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias,
-                                void *y, int y_is_fp32, int M, int N, int K, int unpack, int max_ctas, void *ws,
-                                size_t ws_bytes, void *stream);
-/* Workspace bytes of the K-split tensor-core GEMV (0 when it does not apply to K). */
-I4_API size_t i4_int4_gemv_ksplit_ws_bytes(int N, int K);
+                                void *y, int y_is_fp32, int M, int N, int K, int unpack, int max_ctas, void *stream);
 
 #ifdef __cplusplus
 }

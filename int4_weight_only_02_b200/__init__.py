@@ -64,8 +64,7 @@ _SIGS = {
     "i4_last_error": (ctypes.c_char_p, []),
     "i4_version": (ctypes.c_char_p, []),
     "int4_gemv": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
-    "i4_int4_gemv_variant": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
-    "i4_int4_gemv_ksplit_ws_bytes": (_sz, [_i, _i]),
+    "i4_int4_gemv_variant": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "i4_int4_unpack": (_i, [_vp, _vp, _i, _i, _vp]),
     "paged_gqa_decode_ws_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "paged_gqa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
@@ -137,7 +136,7 @@ def set_option(name: str, value: int):
 # ------------------------------------------------------------------ kernels
 
 def int4_gemv(w, scales, x, bias=None, y=None, out_fp32: bool = False, group: int = 128, stream=None,
-              unpack: int | None = None, max_ctas: int = 0, ws=None):
+              unpack: int | None = None, max_ctas: int = 0):
     """y[M][N] = x[M][K] . dequant(w, scales)^T (+ bias), fp32 accumulation."""
     import torch
     x2 = x if x.dim() == 2 else x.view(1, -1)
@@ -145,19 +144,14 @@ def int4_gemv(w, scales, x, bias=None, y=None, out_fp32: bool = False, group: in
     N = w.shape[0]
     if y is None:
         y = torch.empty((M, N), device=x.device, dtype=torch.float32 if out_fp32 else torch.float16)
-    if unpack is None and max_ctas == 0 and ws is None:
+    if unpack is None and max_ctas == 0:
         st = lib().int4_gemv(_p(w), _p(scales), _p(x2), _p(bias), _p(y), int(out_fp32), M, N, K, group,
                              _stream(stream))
     else:
         st = lib().i4_int4_gemv_variant(_p(w), _p(scales), _p(x2), _p(bias), _p(y), int(out_fp32), M, N, K,
-                                        0 if unpack is None else unpack, max_ctas, _p(ws),
-                                        0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+                                        0 if unpack is None else unpack, max_ctas, _stream(stream))
     _check(st, "int4_gemv")
     return y if x.dim() == 2 else y.view(-1)
-
-
-def int4_gemv_ksplit_ws_bytes(N: int, K: int) -> int:
-    return int(lib().i4_int4_gemv_ksplit_ws_bytes(N, K))
 
 
 def int4_unpack(w, K: int, stream=None):

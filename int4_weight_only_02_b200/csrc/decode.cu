@@ -46,8 +46,6 @@ struct i4_graph {
     unsigned *arrive = nullptr;
     char *attn_ws = nullptr;
     AttnWs attn_layout = {};
-    unsigned *down_cnt = nullptr;   // K-split GEMV of the down projection: arrival counters
-    float *down_part = nullptr;     // and fp32 partial sums
     cudaStream_t cap = nullptr;
     cudaGraph_t graph = nullptr;
     cudaGraphExec_t exec = nullptr;
@@ -153,8 +151,6 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
             a.M = 1;
             a.x = g->mlp;
             a.y = g->resid;
-            a.tile_cnt = g->down_cnt;
-            a.part_ws = g->down_part;
             if (!skip() && (st_ = launch_gemv(PRO_PLAIN, EPI_RESID, a, st, pdl(), g->unpack, 0))) return st_;
             ++n;
         }
@@ -277,8 +273,6 @@ extern "C" int decode_step_graph_create(const i4_model_desc *desc, const i4_mode
     const size_t o_rope = off; off += a256((size_t)desc->max_ctx * (D / 2) * sizeof(float2));
     const size_t o_best = off; off += 256;
     const size_t o_attn_ws = off; off += a256(g->attn_layout.bytes);
-    const size_t down_ws = ksplit_ws_bytes(desc->hidden, desc->intermediate);
-    const size_t o_down = off; off += a256(down_ws);
     if (cudaMalloc(&g->ws, off) != cudaSuccess) {
         cudaGetLastError();
         release(g);
@@ -292,11 +286,6 @@ extern "C" int decode_step_graph_create(const i4_model_desc *desc, const i4_mode
     g->best = reinterpret_cast<unsigned long long *>(g->ws + o_best);
     g->arrive = reinterpret_cast<unsigned *>(g->ws + o_best + 8);
     g->attn_ws = g->ws + o_attn_ws;
-    if (down_ws) {
-        const size_t cnt = ((size_t)(desc->hidden + 15) / 16 * sizeof(unsigned) + 255) & ~(size_t)255;
-        g->down_cnt = reinterpret_cast<unsigned *>(g->ws + o_down);
-        g->down_part = reinterpret_cast<float *>(g->ws + o_down + cnt);
-    }
 
     if ((st = cuda_check(cudaStreamCreateWithFlags(&g->cap, cudaStreamNonBlocking), "stream create")) ||
         (st = cuda_check(cudaMemsetAsync(g->ws, 0, off, g->cap), "workspace clear")) ||
@@ -366,12 +355,17 @@ extern "C" int i4_set_option(const char *name, int value) {
         return I4_OK;
     }
     if (n == "unpack") {
-        if (value < UNPACK_EXACT || value > UNPACK_MMA) return fail(I4_EINVAL, "unpack must be 0, 1, 2 or 3");
+        if (value < UNPACK_EXACT || value > UNPACK_AUTO) return fail(I4_EINVAL, "unpack must be 0, 1, 2, 3 or 4");
         g_default_unpack = value;
         return I4_OK;
     }
     if (n == "stream") {
         set_stream_options(value, 0);
+        return I4_OK;
+    }
+    if (n == "gemv_ctas_per_sm") {
+        if (value < 1 || value > 2) return fail(I4_EINVAL, "gemv_ctas_per_sm must be 1 or 2");
+        set_stream_ctas_per_sm(value);
         return I4_OK;
     }
     if (n == "stream_smem_kb") {

@@ -170,10 +170,11 @@ static int launch_gemv_u(const GemvArgs &a, cudaStream_t stream, bool pdl, int u
     return launch_gemv_mr<PRO, EPI, UNPACK_EXACT>(a, stream, pdl, max_ctas);
 }
 
-int g_default_unpack = UNPACK_EXACT;
+int g_default_unpack = UNPACK_AUTO;
 
 int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool pdl, int unp, int max_ctas) {
     if (unp < 0) unp = g_default_unpack;
+    if (unp == UNPACK_AUTO) unp = a.M == 1 ? UNPACK_MMA : UNPACK_EXACT;
     StreamGeom geo;
     if (max_ctas == 0 && stream_geometry(epi, a, geo, unp)) return launch_gemv_stream(pro, epi, a, geo, stream, pdl, unp);
     if (max_ctas == 0 && unp == UNPACK_MMA && stream_geometry(epi, a, geo, UNPACK_SUBNORMAL))
@@ -198,8 +199,7 @@ int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool p
 using namespace i4;
 
 static int gemv_entry(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
-                      int y_is_fp32, int M, int N, int K, int group, int unp, int max_ctas, cudaStream_t stream,
-                      void *ws = nullptr, size_t ws_bytes = 0) {
+                      int y_is_fp32, int M, int N, int K, int group, int unp, int max_ctas, cudaStream_t stream) {
     if (!w || !scales || !x || !y) return fail(I4_EINVAL, "int4_gemv: null pointer");
     if (group != 128) return fail(I4_EUNSUPPORTED, "int4_gemv: group must be 128 (got %d)", group);
     if (K <= 0 || K % 128 != 0 || K > 32768)
@@ -221,15 +221,6 @@ static int gemv_entry(const uint32_t *w, const uint16_t *scales, const uint16_t 
     a.M = M;
     a.bias = bias;
     a.y = y;
-    if (ws) {
-        const size_t need = ksplit_ws_bytes(N, K);
-        if (!need) return fail(I4_EUNSUPPORTED, "int4_gemv: no K-split kernel for K=%d", K);
-        if (ws_bytes < need || !aligned(ws, 256))
-            return fail(I4_EINVAL, "int4_gemv: K-split workspace of %zu bytes (256-aligned) needed", need);
-        const size_t cnt = ((size_t)(N + 15) / 16 * sizeof(unsigned) + 255) & ~(size_t)255;
-        a.tile_cnt = reinterpret_cast<unsigned *>(ws);
-        a.part_ws = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + cnt);
-    }
     return launch_gemv(PRO_PLAIN, y_is_fp32 ? EPI_F32 : EPI_F16, a, stream, false, unp, max_ctas);
 }
 
@@ -242,13 +233,10 @@ extern "C" int int4_gemv(const uint32_t *w, const uint16_t *scales, const uint16
 // (0 = none); used by the tests and the benchmark to compare variants.
 extern "C" int i4_int4_gemv_variant(const uint32_t *w, const uint16_t *scales, const uint16_t *x,
                                     const uint16_t *bias, void *y, int y_is_fp32, int M, int N, int K, int unpack,
-                                    int max_ctas, void *ws, size_t ws_bytes, void *stream) {
-    if (unpack < UNPACK_EXACT || unpack > UNPACK_MMA) return fail(I4_EINVAL, "unknown unpack variant");
-    return gemv_entry(w, scales, x, bias, y, y_is_fp32, M, N, K, 128, unpack, max_ctas, (cudaStream_t)stream, ws,
-                      ws_bytes);
+                                    int max_ctas, void *stream) {
+    if (unpack < UNPACK_EXACT || unpack > UNPACK_AUTO) return fail(I4_EINVAL, "unknown unpack variant");
+    return gemv_entry(w, scales, x, bias, y, y_is_fp32, M, N, K, 128, unpack, max_ctas, (cudaStream_t)stream);
 }
-
-extern "C" size_t i4_int4_gemv_ksplit_ws_bytes(int N, int K) { return N > 0 && K > 0 ? ksplit_ws_bytes(N, K) : 0; }
 
 extern "C" int i4_int4_unpack(const uint32_t *w, int8_t *q, int N, int K, void *stream) {
     if (!w || !q) return fail(I4_EINVAL, "i4_int4_unpack: null pointer");

@@ -10,7 +10,9 @@ constexpr int kGemvWarps = kGemvThreads / 32;
 
 enum GemvPrologue : int { PRO_PLAIN = 0, PRO_RMSNORM = 1, PRO_EMBED = 2 };
 enum GemvEpilogue : int { EPI_F16 = 0, EPI_F32 = 1, EPI_RESID = 2, EPI_ROPE_KV = 3, EPI_SILU = 4, EPI_ARGMAX = 5 };
-enum GemvUnpack : int { UNPACK_EXACT = 0, UNPACK_SUBNORMAL = 1, UNPACK_MAGIC32 = 2, UNPACK_MMA = 3 };
+// UNPACK_AUTO picks per launch: the tensor-core kernel for single-vector GEMVs (the fastest whole decode
+// step measured), the exact CUDA-core unpack for M > 1.
+enum GemvUnpack : int { UNPACK_EXACT = 0, UNPACK_SUBNORMAL = 1, UNPACK_MAGIC32 = 2, UNPACK_MMA = 3, UNPACK_AUTO = 4 };
 
 struct GemvArgs {
     const uint32_t *w;
@@ -42,8 +44,6 @@ struct GemvArgs {
     int n_prompt;
     // K-split tensor-core kernel: fp32 partial sums [tiles][kslices][16] and one
     // arrival counter per 16-row tile (zero before the first use, left zero)
-    float *part_ws;
-    unsigned *tile_cnt;
 };
 
 size_t gemv_smem_bytes(int K, int mr, int unp);
@@ -58,12 +58,12 @@ struct StreamGeom {
 };
 // Workspace bytes of the K-split tensor-core GEMV for N rows and reduction length K
 // (0 when that kernel does not apply); counters first, then partial sums.
-size_t ksplit_ws_bytes(int N, int K);
 // False when the shape or alignment does not fit the streaming kernel.
 bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp);
 int launch_gemv_stream(int pro, int epi, const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl,
                        int unp);
 void set_stream_options(int enabled, int smem_kb);
+void set_stream_ctas_per_sm(int n);
 // unp < 0 selects the library default; max_ctas <= 0 means no cap.
 int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool pdl, int unp, int max_ctas);
 

@@ -476,6 +476,112 @@ __device__ __forceinline__ void epilogue(const GemvArgs &a, int p, int ra, int r
     }
 }
 
+// Epilogue inputs read from global memory, loaded at the start of a tile so their
+// latency hides under the tile's arithmetic (the residual of EPI_RESID, the bias
+// and cos/sin of EPI_ROPE_KV, the bias of EPI_F16/EPI_F32).
+struct EpiIn {
+    float a, b;
+    float2 cs;
+};
+
+// Per-CTA constants of EPI_ROPE_KV: the position and its page (read once, after the dependency wait).
+struct EpiCta {
+    int pos, page;
+};
+
+template <int EPI>
+__device__ __forceinline__ EpiCta epi_cta(const GemvArgs &a) {
+    EpiCta c = {0, 0};
+    if constexpr (EPI == EPI_ROPE_KV) {
+        c.pos = *a.pos;
+        if (c.pos >= 0 && c.pos < a.max_ctx) c.page = a.page_table[c.pos / a.page_size];
+    }
+    return c;
+}
+
+template <int EPI>
+__device__ __forceinline__ EpiIn epi_load(const GemvArgs &a, int p, int ra, int rb, const EpiCta &c) {
+    EpiIn e = {0.f, 0.f, make_float2(0.f, 0.f)};
+    if constexpr (EPI == EPI_RESID) {
+        const uint16_t *r = reinterpret_cast<const uint16_t *>(a.y);
+        e.a = half_bits_to_float(r[ra]);
+        if (rb >= 0) e.b = half_bits_to_float(r[rb]);
+    } else if constexpr (EPI == EPI_ROPE_KV) {
+        e.a = half_bits_to_float(a.bias[ra]);
+        e.b = half_bits_to_float(a.bias[rb]);
+        if (c.pos >= 0 && c.pos < a.max_ctx && (p >> 6) < a.n_q + a.n_kv) e.cs = a.rope_cs[(size_t)c.pos * 64 + (p & 63)];
+    } else if constexpr (EPI == EPI_F16 || EPI == EPI_F32) {
+        if (a.bias) {
+            e.a = half_bits_to_float(a.bias[ra]);
+            if (rb >= 0) e.b = half_bits_to_float(a.bias[rb]);
+        }
+    }
+    return e;
+}
+
+// epilogue<EPI, 1> with the inputs already loaded (same arithmetic, same stores)
+template <int EPI>
+__device__ __forceinline__ void epilogue_in(const GemvArgs &a, int p, int ra, int rb, float va, float vb,
+                                            const EpiIn &e, const EpiCta &c, unsigned long long &best) {
+    if constexpr (EPI == EPI_F16 || EPI == EPI_F32) {
+        if (a.bias) {
+            va += e.a;
+            vb += e.b;
+        }
+        if constexpr (EPI == EPI_F16) {
+            uint16_t *y = reinterpret_cast<uint16_t *>(a.y);
+            y[ra] = float_to_half_bits(va);
+            if (rb >= 0) y[rb] = float_to_half_bits(vb);
+        } else {
+            float *y = reinterpret_cast<float *>(a.y);
+            y[ra] = va;
+            if (rb >= 0) y[rb] = vb;
+        }
+    } else if constexpr (EPI == EPI_RESID) {
+        uint16_t *r = reinterpret_cast<uint16_t *>(a.y);
+        r[ra] = float_to_half_bits(e.a + rnd16(va));
+        if (rb >= 0) r[rb] = float_to_half_bits(e.b + rnd16(vb));
+    } else if constexpr (EPI == EPI_SILU) {
+        reinterpret_cast<uint16_t *>(a.y)[p] = silu_mul_bits(rnd16(va), rnd16(vb));
+    } else if constexpr (EPI == EPI_ROPE_KV) {
+        const int head = p >> 6, i = p & 63;
+        const float xa = rnd16(va + e.a);
+        const float xb = rnd16(vb + e.b);
+        if (c.pos < 0 || c.pos >= a.max_ctx) {
+            if (a.status) *a.status = 2;
+            return;
+        }
+        if (head < a.n_q + a.n_kv) {
+            uint16_t oa, ob;
+            rope_pair(xa, xb, e.cs, oa, ob);
+            if (head < a.n_q) {
+                a.q_out[head * 128 + i] = oa;
+                a.q_out[head * 128 + i + 64] = ob;
+            } else {
+                const int g = head - a.n_q;
+                const size_t off = (((size_t)c.page * a.n_kv + g) * a.page_size + c.pos % a.page_size) * 128;
+                a.k_pool[off + i] = oa;
+                a.k_pool[off + i + 64] = ob;
+            }
+        } else {
+            const int g = head - a.n_q - a.n_kv;
+            const size_t off = (((size_t)c.page * a.n_kv + g) * a.page_size + c.pos % a.page_size) * 128;
+            a.v_pool[off + i] = float_to_half_bits(xa);
+            a.v_pool[off + i + 64] = float_to_half_bits(xb);
+        }
+    } else if constexpr (EPI == EPI_ARGMAX) {
+        float *lg = reinterpret_cast<float *>(a.y);
+        lg[ra] = va;
+        unsigned long long k = argmax_key(va, ra);
+        best = k > best ? k : best;
+        if (rb >= 0) {
+            lg[rb] = vb;
+            k = argmax_key(vb, rb);
+            best = k > best ? k : best;
+        }
+    }
+}
+
 // Last CTA of the lm_head GEMV: pick the token and advance the sequence state.
 __device__ __forceinline__ void finish_step(const GemvArgs &a, unsigned long long cta_best) {
     __shared__ unsigned long long sbest[32];

@@ -249,89 +249,92 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_stream_kernel(const Ge
 
 // ---------------------------------------------------------------- tensor-core consumer (UNPACK_MMA)
 //
-// Same ring, same tiles of 16 rows (K <= 4096), but the multiply-accumulate runs
-// on mma.sync.m16n8k16 (fp16 in, fp32 accumulate): the 16 weight rows of a
-// tile are the A operand, x (the same vector in all 8 columns of B) the B
-// operand. The unpack is the LOP3 subnormal one (u = q + 8 as u * 2^-24, or
-// 16u * 2^-24 for the high field of each byte), so low and high fields feed two
-// accumulators; per group of 128 k a warp folds them with the row's scale:
-//   y += s * ((lo + hi/16) * 2^24 - 8 * sum_group(x)).
-// Seven consumer warps split the tile's groups evenly; their row sums meet in
-// shared memory and eight threads run the pair epilogues. Rows are placed
-// kMmaRowPad bytes apart in shared memory (one bulk copy per row) so the
-// 16-byte fragment loads of two rows never hit the same banks.
-constexpr int kMmaWarps = 7;
-constexpr int kMmaConsumers = kMmaWarps * 32;
-constexpr int kMmaThreads = kMmaConsumers + 32;
-constexpr int kMmaRowPad = 64;
+// Same producer, ring and tiles as above (whole rows, one bulk copy per tile
+// stream), but the multiply-accumulate runs on mma.sync.m16n8k16 (fp16 in,
+// fp32 accumulate) and one MMA consumes 256 weights:
+//   * a warp works on a row pair (r, r'): A rows 0-7 hold row r, rows 8-15 row r';
+//   * lane (g, c) = (lane / 4, lane % 4) reads 16 contiguous bytes of each row
+//     (32 weights), so one 16-byte load instruction covers 512 contiguous bytes
+//     of one row and never conflicts on shared-memory banks; a block is the
+//     1024 weights one such load covers, and lane (g, c) of block b holds
+//     k = 1024 b + 32 (4 g + c) .. + 31, all inside group 8 b + g;
+//   * the lane's A fragment is its own weights (subnormal LOP3 unpack: low
+//     fields u * 2^-24 into the "lo" MMA, high fields 16 u * 2^-24 into the
+//     "hi" MMA) and its B fragment the x values at the same k, so B column g is
+//     fed only by lanes (g, *): D[g][g] is row r's dot product over group 8b+g
+//     and D[g+8][g] row r''s. Lane (g, g / 2) holds both; the other D entries
+//     mix groups and are never read;
+//   * per block and row: y += s * ((lo + hi / 16) * 2^24 - 8 * sum_group(x)).
+// x is staged once per CTA in lane order (per block, word and lane one 16-byte
+// entry: x pairs (0,4) (2,6) for the lo MMA, (1,5) (3,7) for the hi MMA), so a lane's four B loads per block are
+// 16-byte loads of consecutive lanes. Long rows (K > 4096) use 2-row tiles
+// whose blocks are split over the 8 consumer warps and summed in shared memory.
+constexpr int kTcBlockK = 1024;
 
-// Shared-memory distance between the rows of a tile: the row bytes rounded up so
-// that consecutive rows start 64 bytes apart modulo 128 (two rows of one
-// 16-byte fragment load then cover all 32 banks once).
-__host__ __device__ constexpr int mma_row_stride(int seg) { return seg + ((64 - (seg & 127) + 128) & 127); }
+__host__ __device__ constexpr int tc_blocks(int K) { return (K + kTcBlockK - 1) / kTcBlockK; }
+// staged x: [block][word 0..3][lane] uint4, then 8 * sum(x) per group (fp32)
+__host__ __device__ constexpr long long tc_x_bytes(int K) { return (long long)tc_blocks(K) * 2048 + (K / 128) * 4; }
 
-__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
     asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <int EPI>
-__device__ __forceinline__ void issue_tile_rows(const GemvArgs &a, int t, unsigned char *stage, int row_stride,
-                                                uint64_t *bar, uint64_t pol) {
-    const int wrow = a.K >> 1, srow = a.K >> 6;
-    int ra0, na, rb0, nb;
-    tile_rows<EPI, 16>(a, t, ra0, na, rb0, nb);
-    mbar_expect_tx(bar, (unsigned)((na + nb) * (wrow + srow)));
-    const unsigned char *w = reinterpret_cast<const unsigned char *>(a.w);
-    const unsigned char *s = reinterpret_cast<const unsigned char *>(a.s);
-    unsigned char *sc = stage + 16 * row_stride;
-    for (int r = 0; r < na; ++r)
-        bulk_load(stage + (size_t)r * row_stride, w + (size_t)(ra0 + r) * wrow, wrow, bar, pol);
-    for (int r = 0; r < nb; ++r)
-        bulk_load(stage + (size_t)(na + r) * row_stride, w + (size_t)(rb0 + r) * wrow, wrow, bar, pol);
-    bulk_load(sc, s + (size_t)ra0 * srow, na * srow, bar, pol);
-    if (nb) bulk_load(sc + na * srow, s + (size_t)rb0 * srow, nb * srow, bar, pol);
+// d = A * B (accumulator starts at zero)
+__device__ __forceinline__ void mma_16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
-// x for the tensor-core consumer: for group j, slot p (0..3) and lane class c
-// (0..3), xm[16j + 4p + c] = pair-permuted word 16j + 4c + p, so the four lane
-// classes read 64 contiguous bytes; sxg[j] = sum of the group's 128 x values.
 template <int PRO, class Group>
-__device__ __forceinline__ void stage_x_mma(const GemvArgs &a, uint4 *xm, float *sxg, float *red, const Group &grp) {
+__device__ __forceinline__ void stage_x_tc(const GemvArgs &a, uint4 *xt, float *sx8, float *red, const Group &grp) {
+    const int nb = tc_blocks(a.K), groups = a.K >> 7;
+    // zero the padding past K (lanes of a partial last block read it)
+    for (int i = (a.K >> 3) + grp.tid(); i < nb * 128; i += grp.size()) {
+        const int b = i >> 7, l = (i & 127) >> 2, w = i & 3;
+        xt[(b * 4 + w) * 32 + l] = make_uint4(0u, 0u, 0u, 0u);
+    }
     for_each_x_word<PRO>(a, red, grp, [&](int wd, uint4 v) {
-        const int j = wd >> 4, c = (wd >> 2) & 3, p = wd & 3;
-        xm[16 * j + 4 * p + c] = permute_pairs(v);
+        const int b = wd >> 7, l = (wd & 127) >> 2, w = wd & 3;
+        const uint4 pp = permute_pairs(v);  // (x0,x4) (x1,x5) (x2,x6) (x3,x7)
+        xt[(b * 4 + w) * 32 + l] = make_uint4(pp.x, pp.z, pp.y, pp.w);
     });
     grp.sync();
-    for (int j = grp.tid(); j < (a.K >> 7); j += grp.size()) {
+    for (int j = grp.tid(); j < groups; j += grp.size()) {
+        const int b = j >> 3, g = j & 7;
         float t = 0.f;
-        for (int i = 0; i < 16; ++i) {
-            const uint4 e = xm[16 * j + i];
-            const uint32_t v[4] = {e.x, e.y, e.z, e.w};
-            for (int q = 0; q < 4; ++q) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&v[q]));
-                t += f.x + f.y;
+        for (int w = 0; w < 4; ++w)
+            for (int c = 0; c < 4; ++c) {
+                const uint4 e = xt[(b * 4 + w) * 32 + 4 * g + c];
+                const uint32_t v[4] = {e.x, e.y, e.z, e.w};
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&v[q]));
+                    t += f.x + f.y;
+                }
             }
-        }
-        sxg[j] = t;
+        sx8[j] = 8.0f * t;
     }
 }
 
-template <int PRO, int EPI>
-__global__ void __launch_bounds__(kMmaThreads, 2) gemv_mma_kernel(const GemvArgs a, const StreamGeom geo) {
+template <int PRO, int EPI, int R>
+__global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvArgs a, const StreamGeom geo) {
+    constexpr int PP = R / 2;               // row pairs per tile
+    constexpr int WP = kConsumerWarps / PP;  // warps per row pair
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kMaxStages];
     __shared__ __align__(8) uint64_t empty[kMaxStages];
     __shared__ float red[32];
-    __shared__ float part[2][kMmaWarps][16];
+    __shared__ float part[2][kConsumerWarps][2];
 
-    const int K = a.K, groups = K >> 7, srow = K >> 6;
-    const int row_stride = mma_row_stride(K >> 1);
+    const int K = a.K, wrow = K >> 1, groups = K >> 7, nb = tc_blocks(K);
     const int S = geo.stages;
     unsigned char *ring = smem;
-    uint4 *xm = reinterpret_cast<uint4 *>(smem + (size_t)S * geo.stage_bytes);
-    float *sxg = reinterpret_cast<float *>(xm + (K >> 3));
+    uint4 *xt = reinterpret_cast<uint4 *>(smem + (size_t)S * geo.stage_bytes);
+    float *sx8 = reinterpret_cast<float *>(xt + (size_t)nb * 128);
     const int t_begin = (int)(((long long)blockIdx.x * geo.tiles) / gridDim.x);
     const int t_end = (int)(((long long)(blockIdx.x + 1) * geo.tiles) / gridDim.x);
     const int n_tiles = t_end - t_begin;
@@ -339,7 +342,7 @@ __global__ void __launch_bounds__(kMmaThreads, 2) gemv_mma_kernel(const GemvArgs
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kMmaWarps);
+            mbar_init(&empty[s], kConsumerWarps);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -347,6 +350,7 @@ __global__ void __launch_bounds__(kMmaThreads, 2) gemv_mma_kernel(const GemvArgs
 
     unsigned long long best = 0ull;
     if (threadIdx.x < 32) {
+        // ---------------- producer: weights do not depend on earlier kernels, so no dependency wait
         if (threadIdx.x == 0) {
             const uint64_t pol = evict_first_policy();
             for (int i = 0; i < n_tiles; ++i) {
@@ -355,77 +359,102 @@ __global__ void __launch_bounds__(kMmaThreads, 2) gemv_mma_kernel(const GemvArgs
                     record_error(&g_device_error, 1);
                     break;
                 }
-                issue_tile_rows<EPI>(a, t_begin + i, ring + (size_t)s * geo.stage_bytes, row_stride, &full[s], pol);
+                issue_tile<EPI, R>(a, t_begin + i, ring + (size_t)s * geo.stage_bytes, &full[s], pol);
             }
         }
     } else {
-        const NamedGroup<32, kMmaConsumers> grp;
+        // ---------------- consumers
+        const NamedGroup<32, kConsumers> grp;
         grid_dep_wait();
-        stage_x_mma<PRO>(a, xm, sxg, red, grp);
+        stage_x_tc<PRO>(a, xt, sx8, red, grp);
         grp.sync();
         grid_dep_launch();
         const int c_id = grp.tid(), warp = c_id >> 5, lane = c_id & 31;
-        const int g = lane >> 2, cl = lane & 3;
-        const int j0 = (warp * groups) / kMmaWarps, j1 = ((warp + 1) * groups) / kMmaWarps;
+        const int g = lane >> 2, c = lane & 3;
+        const bool diag = c == (g >> 1);  // this lane holds D[g][g] and D[g+8][g]
+        const int pr = warp / WP, wp = warp % WP;
+        const int b0 = (wp * nb) / WP, b1 = ((wp + 1) * nb) / WP;
+        const int tra = kPaired<EPI> ? pr : 2 * pr, trb = kPaired<EPI> ? pr + PP : 2 * pr + 1;
+        const EpiCta ecta = epi_cta<EPI>(a);
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
             const int s = i % S, n = i / S, t = t_begin + i;
+            int ra0, na, rb0, nb_rows;
+            tile_rows<EPI, R>(a, t, ra0, na, rb0, nb_rows);
+            // epilogue inputs first: their global-memory latency overlaps the wait and the arithmetic
+            const int p = t * PP + pr;
+            int pa, pb;
+            pair_rows<EPI>(a, p, pa, pb);
+            const bool epi_lane = lane == 0 && wp == 0 && trb < na + nb_rows;
+            EpiIn ein = {0.f, 0.f, make_float2(0.f, 0.f)};
+            if (epi_lane) ein = epi_load<EPI>(a, p, pa, pb, ecta);
             if (ok && !mbar_wait(&full[s], (unsigned)(n & 1))) {
                 record_error(&g_device_error, 1);
                 ok = false;
             }
-            int ra0, na, rb0, nb;
-            tile_rows<EPI, 16>(a, t, ra0, na, rb0, nb);
-            const int rows = na + nb;
-            const unsigned char *st = ring + (size_t)s * geo.stage_bytes;
-            const uint16_t *sc = reinterpret_cast<const uint16_t *>(st + 16 * row_stride);
-            // rows past the tile's end hold stale bytes: their results are never used
-            const unsigned char *wg = st + (size_t)g * row_stride;
-            const unsigned char *wg8 = st + (size_t)(g + 8) * row_stride;
-            float tot_g = 0.f, tot_g8 = 0.f;
-            if (ok) {
-                for (int j = j0; j < j1; ++j) {
-                    const uint4 qa = *reinterpret_cast<const uint4 *>(wg + (size_t)(16 * j + 4 * cl) * 4);
-                    const uint4 qb = *reinterpret_cast<const uint4 *>(wg8 + (size_t)(16 * j + 4 * cl) * 4);
-                    const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
-                    float lo[4] = {0.f, 0.f, 0.f, 0.f}, hi[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const uint4 xc = xm[16 * j + 4 * p + cl];
-                        uint32_t ua[4], ub[4];
-                        unpack_word_subnormal(wa[p], ua);   // (k0,k4) (k1,k5) (k2,k6) (k3,k7)
-                        unpack_word_subnormal(wb[p], ub);
-                        const uint32_t alo[4] = {ua[0], ub[0], ua[2], ub[2]};  // low fields
-                        const uint32_t ahi[4] = {ua[1], ub[1], ua[3], ub[3]};  // high fields (16u)
-                        mma_16816(lo, alo, xc.x, xc.z);
-                        mma_16816(hi, ahi, xc.y, xc.w);
+            const bool live = ok && trb < na + nb_rows;
+            float tot_a = 0.f, tot_b = 0.f;
+            if (live) {
+                const unsigned char *st = ring + (size_t)s * geo.stage_bytes;
+                const unsigned char *wa = st + (size_t)tra * wrow + 16 * lane;
+                const unsigned char *wb = st + (size_t)trb * wrow + 16 * lane;
+                const uint16_t *sa = reinterpret_cast<const uint16_t *>(st + (size_t)R * wrow) + tra * groups;
+                const uint16_t *sb = reinterpret_cast<const uint16_t *>(st + (size_t)R * wrow) + trb * groups;
+#pragma unroll 2
+                for (int b = b0; b < b1; ++b) {
+                    // the lane's 32 weights of each row; past K (partial last block) all-zero codes (u = 0)
+                    const bool in = 1024 * b + 32 * lane < K;
+                    uint4 qa = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u), qb = qa;
+                    if (in) {
+                        qa = *reinterpret_cast<const uint4 *>(wa + 512 * b);
+                        qb = *reinterpret_cast<const uint4 *>(wb + 512 * b);
                     }
-                    const float sx8 = 8.0f * sxg[j];
-                    const float vg = fmaf(hi[0], 0.0625f, lo[0]) * 16777216.0f - sx8;
-                    const float vg8 = fmaf(hi[2], 0.0625f, lo[2]) * 16777216.0f - sx8;
-                    tot_g = fmaf(vg, half_bits_to_float(sc[g * groups + j]), tot_g);
-                    tot_g8 = fmaf(vg8, half_bits_to_float(sc[(g + 8) * groups + j]), tot_g8);
+                    const uint32_t wra[4] = {qa.x, qa.y, qa.z, qa.w}, wrb[4] = {qb.x, qb.y, qb.z, qb.w};
+                    float lo[4], hi[4];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const uint4 xc = xt[(b * 4 + w) * 32 + lane];  // (x0,x4) (x2,x6) (x1,x5) (x3,x7)
+                        uint32_t ua[4], ub[4];
+                        unpack_word_subnormal(wra[w], ua);  // (k0,k4) 16(k1,k5) (k2,k6) 16(k3,k7)
+                        unpack_word_subnormal(wrb[w], ub);
+                        if (w == 0) {  // first MMA of the block: accumulate onto zero
+                            mma_16816_z(lo, ua[0], ub[0], ua[2], ub[2], xc.x, xc.y);
+                            mma_16816_z(hi, ua[1], ub[1], ua[3], ub[3], xc.z, xc.w);
+                        } else {
+                            mma_16816(lo, ua[0], ub[0], ua[2], ub[2], xc.x, xc.y);
+                            mma_16816(hi, ua[1], ub[1], ua[3], ub[3], xc.z, xc.w);
+                        }
+                    }
+                    const int j = 8 * b + g;  // this lane's group
+                    if (diag && j < groups) {
+                        const bool odd = g & 1;
+                        const float la = odd ? lo[1] : lo[0], ha = odd ? hi[1] : hi[0];
+                        const float lb = odd ? lo[3] : lo[2], hb = odd ? hi[3] : hi[2];
+                        const float sxj = sx8[j];
+                        tot_a = fmaf(fmaf(ha, 0.0625f, la) * 16777216.0f - sxj, half_bits_to_float(sa[j]), tot_a);
+                        tot_b = fmaf(fmaf(hb, 0.0625f, lb) * 16777216.0f - sxj, half_bits_to_float(sb[j]), tot_b);
+                    }
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-            if (cl == 0) {
-                part[i & 1][warp][g] = tot_g;
-                part[i & 1][warp][g + 8] = tot_g8;
-            }
-            grp.sync();
-            if (c_id < 8 && ok) {
-                const int tra = kPaired<EPI> ? c_id : 2 * c_id, trb = kPaired<EPI> ? c_id + 8 : 2 * c_id + 1;
-                if (trb < rows) {
+            if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
+            tot_a = warp_sum(tot_a);
+            tot_b = warp_sum(tot_b);
+            if constexpr (WP == 1) {
+                if (epi_lane && live) epilogue_in<EPI>(a, p, pa, pb, tot_a, tot_b, ein, ecta, best);
+            } else {
+                if (lane == 0) {
+                    part[i & 1][warp][0] = tot_a;
+                    part[i & 1][warp][1] = tot_b;
+                }
+                grp.sync();
+                if (epi_lane && live) {
                     float va = 0.f, vb = 0.f;
-                    for (int w = 0; w < kMmaWarps; ++w) {
-                        va += part[i & 1][w][tra];
-                        vb += part[i & 1][w][trb];
+                    for (int w = 0; w < WP; ++w) {
+                        va += part[i & 1][warp + w][0];
+                        vb += part[i & 1][warp + w][1];
                     }
-                    const int p = t * 8 + c_id;
-                    int pa, pb;
-                    pair_rows<EPI>(a, p, pa, pb);
-                    epilogue<EPI, 1>(a, p, pa, pb, &va, &vb, best);
+                    epilogue_in<EPI>(a, p, pa, pb, va, vb, ein, ecta, best);
                 }
             }
         }
@@ -440,225 +469,39 @@ __global__ void __launch_bounds__(kMmaThreads, 2) gemv_mma_kernel(const GemvArgs
     if constexpr (EPI == EPI_ARGMAX) finish_step(a, best);
 }
 
-// ---------------------------------------------------------------- K-split tensor-core consumer
-//
-// For rows too long for whole-row tiles (the MLP down projection, K = 18944):
-// a work unit is one 16-row tile times one of Q slices of K (the smallest Q
-// that divides the groups and keeps a stage near 40 KB; Q = 4 for K = 18944,
-// 37 groups per slice). The producer copies the 16 row segments of the slice
-// plus the tile's whole scale block (its rows are contiguous, so one copy; the
-// per-slice part of a scale row would not be 16-byte aligned). Seven consumer
-// warps run the same mma.sync loop over the slice's groups; the unit's 16 row
-// sums go to a global fp32 workspace and the unit that completes a tile's Q
-// slices (an arrival counter, no waiting) adds them in slice order and runs the
-// epilogue, so results do not depend on timing. One CTA per SM, contiguous
-// unit ranges, four-deep ring.
-constexpr int kKsplitMaxStage = 48 * 1024;
-
-static int ksplit_slices(int K) {
-    const int groups = K / 128, wrow = K / 2;
-    for (int q = 2; q <= 16; ++q) {
-        if (groups % q) continue;
-        const long long stage = 16LL * mma_row_stride(wrow / q) + 16LL * (K / 64);
-        if (stage <= kKsplitMaxStage) return q;
-    }
-    return 0;
-}
-
-size_t ksplit_ws_bytes(int N, int K) {
-    const int q = ksplit_slices(K);
-    if (!q || K <= 32 * kMaxHalvesPerLane * 16) return 0;
-    const size_t tiles = (size_t)(N + 15) / 16;
-    const size_t cnt = (tiles * sizeof(unsigned) + 255) & ~(size_t)255;
-    return cnt + tiles * q * 16 * sizeof(float);
-}
-
-template <int PRO, int EPI>
-__global__ void __launch_bounds__(kMmaThreads, 1) gemv_mma_ksplit_kernel(const GemvArgs a, const StreamGeom geo,
-                                                                         int Q) {
-    extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t full[kMaxStages];
-    __shared__ __align__(8) uint64_t empty[kMaxStages];
-    __shared__ float red[32];
-    __shared__ float part[2][kMmaWarps][16];
-
-    const int K = a.K, groups = K >> 7, srow = K >> 6, wrow = K >> 1;
-    const int GQ = groups / Q, seg = wrow / Q;
-    const int row_stride = mma_row_stride(seg);
-    const int S = geo.stages;
-    unsigned char *ring = smem;
-    uint4 *xm = reinterpret_cast<uint4 *>(smem + (size_t)S * geo.stage_bytes);
-    float *sxg = reinterpret_cast<float *>(xm + (K >> 3));
-    const int u_begin = (int)(((long long)blockIdx.x * geo.tiles) / gridDim.x);
-    const int u_end = (int)(((long long)(blockIdx.x + 1) * geo.tiles) / gridDim.x);
-    const int n_units = u_end - u_begin;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kMmaWarps);
-        }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-
-    if (threadIdx.x < 32) {
-        if (threadIdx.x == 0) {
-            const uint64_t pol = evict_first_policy();
-            const unsigned char *w = reinterpret_cast<const unsigned char *>(a.w);
-            const unsigned char *sg = reinterpret_cast<const unsigned char *>(a.s);
-            for (int i = 0; i < n_units; ++i) {
-                const int s = i % S, n = i / S, u = u_begin + i, t = u / Q, q = u % Q;
-                if (n > 0 && !mbar_wait(&empty[s], (unsigned)((n - 1) & 1))) {
-                    record_error(&g_device_error, 1);
-                    break;
-                }
-                const int r0 = t * 16, rows = (a.N - r0) < 16 ? (a.N - r0) : 16;
-                unsigned char *st = ring + (size_t)s * geo.stage_bytes;
-                mbar_expect_tx(&full[s], (unsigned)(rows * (seg + srow)));
-                for (int r = 0; r < rows; ++r)
-                    bulk_load(st + (size_t)r * row_stride, w + (size_t)(r0 + r) * wrow + (size_t)q * seg, seg, &full[s],
-                              pol);
-                bulk_load(st + 16 * row_stride, sg + (size_t)r0 * srow, rows * srow, &full[s], pol);
-            }
-        }
-    } else {
-        const NamedGroup<32, kMmaConsumers> grp;
-        grid_dep_wait();
-        stage_x_mma<PRO>(a, xm, sxg, red, grp);
-        grp.sync();
-        grid_dep_launch();
-        const int c_id = grp.tid(), warp = c_id >> 5, lane = c_id & 31;
-        const int g = lane >> 2, cl = lane & 3;
-        const int jl0 = (warp * GQ) / kMmaWarps, jl1 = ((warp + 1) * GQ) / kMmaWarps;
-        bool ok = true;
-        unsigned long long best = 0ull;
-        for (int i = 0; i < n_units; ++i) {
-            const int s = i % S, n = i / S, u = u_begin + i, t = u / Q, q = u % Q;
-            if (ok && !mbar_wait(&full[s], (unsigned)(n & 1))) {
-                record_error(&g_device_error, 1);
-                ok = false;
-            }
-            const int r0 = t * 16, rows = (a.N - r0) < 16 ? (a.N - r0) : 16;
-            const unsigned char *st = ring + (size_t)s * geo.stage_bytes;
-            const uint16_t *sc = reinterpret_cast<const uint16_t *>(st + 16 * row_stride);
-            const unsigned char *wg = st + (size_t)g * row_stride;
-            const unsigned char *wg8 = st + (size_t)(g + 8) * row_stride;
-            float tot_g = 0.f, tot_g8 = 0.f;
-            if (ok) {
-                for (int jl = jl0; jl < jl1; ++jl) {
-                    const int j = q * GQ + jl;  // group index along K
-                    const uint4 qa = *reinterpret_cast<const uint4 *>(wg + (size_t)(16 * jl + 4 * cl) * 4);
-                    const uint4 qb = *reinterpret_cast<const uint4 *>(wg8 + (size_t)(16 * jl + 4 * cl) * 4);
-                    const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
-                    float lo[4] = {0.f, 0.f, 0.f, 0.f}, hi[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        const uint4 xc = xm[16 * j + 4 * p + cl];
-                        uint32_t ua[4], ub[4];
-                        unpack_word_subnormal(wa[p], ua);
-                        unpack_word_subnormal(wb[p], ub);
-                        const uint32_t alo[4] = {ua[0], ub[0], ua[2], ub[2]};
-                        const uint32_t ahi[4] = {ua[1], ub[1], ua[3], ub[3]};
-                        mma_16816(lo, alo, xc.x, xc.z);
-                        mma_16816(hi, ahi, xc.y, xc.w);
-                    }
-                    const float sx8 = 8.0f * sxg[j];
-                    const float vg = fmaf(hi[0], 0.0625f, lo[0]) * 16777216.0f - sx8;
-                    const float vg8 = fmaf(hi[2], 0.0625f, lo[2]) * 16777216.0f - sx8;
-                    tot_g = fmaf(vg, half_bits_to_float(sc[g * groups + j]), tot_g);
-                    tot_g8 = fmaf(vg8, half_bits_to_float(sc[(g + 8) * groups + j]), tot_g8);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-            if (cl == 0) {
-                part[i & 1][warp][g] = tot_g;
-                part[i & 1][warp][g + 8] = tot_g8;
-            }
-            grp.sync();
-            if (warp == 0) {
-                // this slice's 16 row sums to the workspace, then count the tile's slices
-                float *pw = a.part_ws + ((size_t)t * Q + q) * 16;
-                if (lane < 16) {
-                    float v = 0.f;
-                    for (int w = 0; w < kMmaWarps; ++w) v += part[i & 1][w][lane];
-                    pw[lane] = v;
-                    __threadfence();
-                }
-                __syncwarp();
-                unsigned prev = 0;
-                if (lane == 0) prev = atomicAdd(a.tile_cnt + t, 1u);
-                prev = __shfl_sync(0xffffffffu, prev, 0);
-                if (prev == (unsigned)Q - 1u && ok) {
-                    __threadfence();
-                    if (lane < 8 && 2 * lane + 1 < rows) {
-                        float va = 0.f, vb = 0.f;
-                        for (int qq = 0; qq < Q; ++qq) {
-                            va += __ldcg(a.part_ws + ((size_t)t * Q + qq) * 16 + 2 * lane);
-                            vb += __ldcg(a.part_ws + ((size_t)t * Q + qq) * 16 + 2 * lane + 1);
-                        }
-                        const int p = t * 8 + lane;
-                        int pa, pb;
-                        pair_rows<EPI>(a, p, pa, pb);
-                        epilogue<EPI, 1>(a, p, pa, pb, &va, &vb, best);
-                    }
-                    if (lane == 0) a.tile_cnt[t] = 0u;  // ready for the next launch
-                }
-            }
-        }
-    }
-}
-
 // ---------------------------------------------------------------- host side
 
 static bool g_stream_enabled = true;
 static int g_stream_smem_budget = 110 * 1024;  // two CTAs per SM
+static int g_stream_ctas_per_sm = 2;
 
 void set_stream_options(int enabled, int smem_kb) {
     if (enabled >= 0) g_stream_enabled = enabled != 0;
     if (smem_kb > 0) g_stream_smem_budget = smem_kb * 1024;
 }
 
+void set_stream_ctas_per_sm(int n) { g_stream_ctas_per_sm = n; }
+
 bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp) {
     if (!g_stream_enabled || a.M != 1 || a.K % 512 != 0 || a.K > 32768 || a.N < 2) return false;
-    if (unp == UNPACK_MMA && a.K > 32 * kMaxHalvesPerLane * 16) {
-        // long rows: K-split tensor-core kernel (plain / fp32 / residual epilogues, needs a workspace)
-        const int Q = ksplit_slices(a.K);
-        if (!Q || !a.part_ws || !a.tile_cnt || a.N % 2 != 0) return false;
-        if (!(epi == EPI_F16 || epi == EPI_F32 || epi == EPI_RESID)) return false;
-        if (!aligned(a.w, 16) || !aligned(a.s, 16)) return false;
-        g.R = -Q;  // marks the K-split kernel; |R| = slices
-        const long long seg = a.K / 2 / Q;
-        g.stage_bytes = (int)((16LL * mma_row_stride((int)seg) + 16 * (a.K / 64) + 127) / 128 * 128);
-        const long long xs_bytes = (long long)a.K * 2 + (long long)(a.K / 128) * 4;
-        int stages = (int)((220 * 1024 - xs_bytes) / g.stage_bytes);
-        if (stages > kMaxStages) stages = kMaxStages;
-        if (stages < 2) return false;
-        g.stages = stages;
-        g.tiles = ((a.N + 15) / 16) * Q;  // work units
-        g.grid = g.tiles < kNumSMs ? g.tiles : kNumSMs;
-        g.tiles_per_cta = (g.tiles + g.grid - 1) / g.grid;
-        g.smem = (int)(stages * (long long)g.stage_bytes + xs_bytes);
-        return true;
-    }
     if (unp == UNPACK_MMA) {
-        if (a.K > 32 * kMaxHalvesPerLane * 16) return false;  // full-row tiles only
         const bool paired = (epi == EPI_SILU || epi == EPI_ROPE_KV);
+        const int R = a.K <= 32 * kMaxHalvesPerLane * 16 ? 16 : 2;
+        if (paired && R != 16) return false;
         if (!paired && a.N % 2 != 0) return false;
-        if (epi == EPI_SILU && a.inter % 8 != 0) return false;
+        if (epi == EPI_SILU && a.inter % (R / 2) != 0) return false;
         if (!aligned(a.w, 16) || !aligned(a.s, 16)) return false;
-        g.R = 16;
-        const long long row_stride = mma_row_stride(a.K / 2);
-        g.stage_bytes = (int)((16 * row_stride + 16 * (a.K / 64) + 127) / 128 * 128);
-        const long long xs_bytes = (long long)a.K * 2 + (long long)(a.K / 128) * 4;
+        const long long wrow = a.K / 2, srow = a.K / 64;
+        g.R = R;
+        g.stage_bytes = (int)(((R * (wrow + srow)) + 127) / 128 * 128);
+        const long long xs_bytes = (tc_x_bytes(a.K) + 127) / 128 * 128;
         int stages = (int)((g_stream_smem_budget - xs_bytes) / g.stage_bytes);
         if (stages > kMaxStages) stages = kMaxStages;
         if (stages < 2) return false;
         g.stages = stages;
         const long long pairs = (epi == EPI_SILU) ? a.inter : (long long)(a.N / 2);
-        g.tiles = paired ? (int)(pairs / 8) : (a.N + 15) / 16;
-        g.grid = g.tiles < 2 * kNumSMs ? g.tiles : 2 * kNumSMs;
+        g.tiles = paired ? (int)(pairs / (R / 2)) : (a.N + R - 1) / R;
+        g.grid = g.tiles < g_stream_ctas_per_sm * kNumSMs ? g.tiles : g_stream_ctas_per_sm * kNumSMs;
         g.tiles_per_cta = (g.tiles + g.grid - 1) / g.grid;
         g.smem = (int)(stages * (long long)g.stage_bytes + xs_bytes);
         return true;
@@ -681,7 +524,7 @@ bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp) {
     g.stages = stages;
     const long long pairs = (epi == EPI_SILU) ? a.inter : (long long)(a.N / 2);
     g.tiles = paired ? (int)(pairs / (R / 2)) : (a.N + R - 1) / R;
-    g.grid = g.tiles < 2 * kNumSMs ? g.tiles : 2 * kNumSMs;
+    g.grid = g.tiles < g_stream_ctas_per_sm * kNumSMs ? g.tiles : g_stream_ctas_per_sm * kNumSMs;
     g.tiles_per_cta = (g.tiles + g.grid - 1) / g.grid;
     g.smem = (int)(stages * (long long)g.stage_bytes + xs_bytes);
     return true;
@@ -711,38 +554,28 @@ static int launch_stream_r(const GemvArgs &a, const StreamGeom &geo, cudaStream_
     }
 }
 
-template <int PRO, int EPI>
-static int launch_ksplit_t(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
-    if constexpr (EPI == EPI_F16 || EPI == EPI_F32 || EPI == EPI_RESID) {
-        auto kern = gemv_mma_ksplit_kernel<PRO, EPI>;
-        static int configured = -1;
-        if (geo.smem > configured) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, geo.smem);
-            if (e != cudaSuccess) return cuda_check(e, "k-split gemv smem attribute");
-            configured = geo.smem;
-        }
-        if (g_dry_run) return I4_OK;
-        return cuda_check(
-            launch(kern, dim3(geo.grid), dim3(kMmaThreads), (size_t)geo.smem, stream, pdl, a, geo, -geo.R),
-            "k-split gemv launch");
-    } else {
-        return fail(I4_EUNSUPPORTED, "k-split gemv: epilogue not supported");
+template <int PRO, int EPI, int R>
+static int launch_tc_t(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
+    auto kern = gemv_tc_kernel<PRO, EPI, R>;
+    static int configured = -1;
+    if (geo.smem > configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, geo.smem);
+        if (e != cudaSuccess) return cuda_check(e, "tensor-core gemv smem attribute");
+        configured = geo.smem;
     }
+    if (g_dry_run) return I4_OK;
+    return cuda_check(launch(kern, dim3(geo.grid), dim3(kStreamThreads), (size_t)geo.smem, stream, pdl, a, geo),
+                      "tensor-core gemv launch");
 }
 
 template <int PRO, int EPI>
 static int launch_mma_t(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
-    if (geo.R < 0) return launch_ksplit_t<PRO, EPI>(a, geo, stream, pdl);
-    auto kern = gemv_mma_kernel<PRO, EPI>;
-    static int configured = -1;
-    if (geo.smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, geo.smem);
-        if (e != cudaSuccess) return cuda_check(e, "mma gemv smem attribute");
-        configured = geo.smem;
+    if (geo.R == 16) return launch_tc_t<PRO, EPI, 16>(a, geo, stream, pdl);
+    if constexpr (EPI == EPI_SILU || EPI == EPI_ROPE_KV) {
+        return fail(I4_EUNSUPPORTED, "tensor-core gemv: paired epilogue needs 16-row tiles");
+    } else {
+        return launch_tc_t<PRO, EPI, 2>(a, geo, stream, pdl);
     }
-    if (g_dry_run) return I4_OK;
-    return cuda_check(launch(kern, dim3(geo.grid), dim3(kMmaThreads), (size_t)geo.smem, stream, pdl, a, geo),
-                      "mma gemv launch");
 }
 
 template <int PRO, int EPI>

@@ -120,20 +120,15 @@ def test_bad_arguments_raise(i4lib, cuda):
         i4lib.int4_gemv(wd, sd, torch.zeros((9, 256), dtype=torch.float16, device=cuda))
 
 
-@pytest.mark.parametrize("n,k", [(3584, 18944), (64, 4608), (30, 8192)])
-def test_ksplit_tensor_core_kernel(i4lib, cuda, n, k):
-    """Rows too long for whole-row tiles: the K-split mma.sync kernel with its workspace."""
+@pytest.mark.parametrize("n,k", [(3584, 18944), (64, 4608), (30, 8192), (6, 2560), (14, 1536)])
+def test_tensor_core_kernel_block_edges(i4lib, cuda, n, k):
+    """The tensor-core kernel on long rows (2-row tiles, blocks split over warps) and on K that
+    ends inside a 1024-weight block (18944, 2560 and 1536 leave half or a quarter of a block)."""
     import torch
     w, s, x, b = synth.gemv_case(n, k, seed=9, bias=True)
     ref = oracle.int4_gemv(w, s, x[0], b)
-    nbytes = i4lib.int4_gemv_ksplit_ws_bytes(n, k)
-    assert nbytes > 0
-    ws = torch.zeros(nbytes, dtype=torch.uint8, device=cuda)
     args = [dev(a, cuda) for a in (w, s, x)]
-    for _ in range(2):  # the counters must come back to zero for the second call
-        got = i4lib.int4_gemv(*args, bias=dev(b, cuda), unpack=3, ws=ws)
-        torch.cuda.synchronize()
-        assert normwise_err(got.cpu().numpy()[0], ref) <= TOL
-    cnt = ((n + 15) // 16 * 4 + 255) // 256 * 256
-    assert int(ws[:cnt].sum().item()) == 0
+    got = i4lib.int4_gemv(*args, bias=dev(b, cuda), unpack=3)
+    torch.cuda.synchronize()
+    assert normwise_err(got.cpu().numpy()[0], ref) <= TOL
     assert i4lib.device_error() == 0
