@@ -235,6 +235,8 @@ def run_profile_kernel(args):
         i4.set_option("unpack", args.unpack)
     if args.gemv_ctas is not None:
         i4.set_option("gemv_ctas_per_sm", args.gemv_ctas)
+    if args.l2_prefetch is not None:
+        i4.set_option("l2_prefetch", args.l2_prefetch)
     shape = synth.ModelShape(layers=1)
     dev = torch.device("cuda", 0)
     layers = [synth.layer_weights(synth.QWEN7B, 0, 0)]
@@ -350,6 +352,7 @@ def main():
     ap.add_argument("--pdl", type=int, default=None, help="override programmatic dependent launch (0/1)")
     ap.add_argument("--unpack", type=int, default=None, help="override the GEMV unpack variant (0..4, 4 = per shape)")
     ap.add_argument("--gemv-ctas", type=int, default=None, help="override the GEMV CTAs per SM (1 or 2)")
+    ap.add_argument("--l2-prefetch", type=int, default=None, help="override the next-GEMV L2 prefetch (0/1)")
     ap.add_argument("--profile-kernel", default=None, choices=sorted(PROFILE_KERNELS),
                     help="profiling mode: a one-layer model of the same shapes, then only this kernel of the "
                          "decode step, --launches times (for ncu captures)")
@@ -391,6 +394,8 @@ def main():
         i4.set_option("unpack", args.unpack)
     if args.gemv_ctas is not None:
         i4.set_option("gemv_ctas_per_sm", args.gemv_ctas)
+    if args.l2_prefetch is not None:
+        i4.set_option("l2_prefetch", args.l2_prefetch)
 
     shape = synth.QWEN7B
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline

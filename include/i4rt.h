@@ -273,7 +273,9 @@ I4_API int decode_step_launch_kernel(i4_graph *g, int index, void *stream);
  *   "stream" 0/1: use the bulk-copy pipelined GEMV where the shape allows it
  *            (M == 1, K % 512 == 0, 16-byte aligned w and scales), default 1;
  *   "stream_smem_kb" 32..227: shared memory budget of that kernel's ring;
- *   "gemv_ctas_per_sm" 1/2 (default 2): CTAs per SM of the pipelined GEMV grids.
+ *   "gemv_ctas_per_sm" 1/2 (default 2): CTAs per SM of the pipelined GEMV grids;
+ *   "l2_prefetch" 0/1 (default 0): in a decode step, each GEMV prefetches the
+ *            next GEMV's weights into L2 (up to 48 MB) once its own ring is full.
  * Not thread-safe; set options before creating graphs.
  */
 I4_API int i4_set_option(const char *name, int value);

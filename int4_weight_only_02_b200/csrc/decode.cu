@@ -27,8 +27,10 @@
 
 namespace i4 {
 int launch_rope_table(float2 *cs, int max_ctx, int d, double theta, cudaStream_t stream);
+extern bool g_l2_prefetch;
 bool g_dry_run = false;
 bool g_pdl = true;
+bool g_l2_prefetch = false;
 }  // namespace i4
 
 using namespace i4;
@@ -50,6 +52,7 @@ struct i4_graph {
     cudaGraph_t graph = nullptr;
     cudaGraphExec_t exec = nullptr;
     bool pdl = false;
+    bool l2pf = false;  // each GEMV prefetches the next GEMV's weights into L2
     int unpack = UNPACK_EXACT;
     int n_kernels = 0;
 };
@@ -62,6 +65,15 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
     int n = 0, st_ = 0;
     auto pdl = [&]() { return g->pdl && n > 0 && only < 0; };
     auto skip = [&]() { return only >= 0 && only != n; };
+    // L2 prefetch target of a GEMV: the weights and scales of the GEMV that follows it
+    auto prefetch = [&](GemvArgs &a, const uint32_t *w, const uint16_t *sc, int rows, int k) {
+        if (!g->l2pf || only >= 0) return;
+        const size_t cap = 48u << 20;  // a share of L2 the streaming kernels leave alone
+        a.pf_a = w;
+        a.pf_a_bytes = (size_t)rows * (k / 2) < cap ? (size_t)rows * (k / 2) : cap;
+        a.pf_b = sc;
+        a.pf_b_bytes = (size_t)rows * (k / 64);
+    };
     for (int l = 0; l < d.n_layers; ++l) {
         const i4_layer_weights &L = g->layers[l];
         {  // qkv + RoPE + KV append
@@ -89,6 +101,7 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
             a.page_size = d.page_size;
             a.max_ctx = d.max_ctx;
             a.status = g->seq.status;
+            prefetch(a, L.w_o, L.s_o, H, d.n_q_heads * D);
             if (!skip() && (st_ = launch_gemv(l == 0 ? PRO_EMBED : PRO_RMSNORM, EPI_ROPE_KV, a, st, pdl(), g->unpack, 0))) return st_;
             ++n;
         }
@@ -124,6 +137,7 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
             a.M = 1;
             a.x = g->attn;
             a.y = g->resid;
+            prefetch(a, L.w_gate_up, L.s_gate_up, 2 * I, H);
             if (!skip() && (st_ = launch_gemv(PRO_PLAIN, EPI_RESID, a, st, pdl(), g->unpack, 0))) return st_;
             ++n;
         }
@@ -139,6 +153,7 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
             a.eps = d.rms_eps;
             a.y = g->mlp;
             a.inter = I;
+            prefetch(a, L.w_down, L.s_down, H, I);
             if (!skip() && (st_ = launch_gemv(PRO_RMSNORM, EPI_SILU, a, st, pdl(), g->unpack, 0))) return st_;
             ++n;
         }
@@ -151,6 +166,10 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
             a.M = 1;
             a.x = g->mlp;
             a.y = g->resid;
+            if (l + 1 < d.n_layers)
+                prefetch(a, g->layers[l + 1].w_qkv, g->layers[l + 1].s_qkv, nqkv, H);
+            else
+                prefetch(a, g->w.w_lm, g->w.s_lm, d.vocab, H);
             if (!skip() && (st_ = launch_gemv(PRO_PLAIN, EPI_RESID, a, st, pdl(), g->unpack, 0))) return st_;
             ++n;
         }
@@ -261,6 +280,7 @@ extern "C" int decode_step_graph_create(const i4_model_desc *desc, const i4_mode
     g->seq.k_pools = g->kp.data();
     g->seq.v_pools = g->vp.data();
     g->pdl = g_pdl;
+    g->l2pf = g_l2_prefetch;
     g->unpack = g_default_unpack;
 
     const int H = desc->hidden, D = desc->head_dim;
@@ -361,6 +381,10 @@ extern "C" int i4_set_option(const char *name, int value) {
     }
     if (n == "stream") {
         set_stream_options(value, 0);
+        return I4_OK;
+    }
+    if (n == "l2_prefetch") {
+        g_l2_prefetch = value != 0;
         return I4_OK;
     }
     if (n == "gemv_ctas_per_sm") {

@@ -42,8 +42,10 @@ struct GemvArgs {
     int32_t *token_io, *pos_io, *ctx_io, *history, *status;
     const int32_t *prompt;
     int n_prompt;
-    // K-split tensor-core kernel: fp32 partial sums [tiles][kslices][16] and one
-    // arrival counter per 16-row tile (zero before the first use, left zero)
+    // L2 prefetch of the next kernel's weights and scales (bulk prefetch split over
+    // the CTAs, issued once the ring is first filled); null pointers = none
+    const void *pf_a, *pf_b;
+    size_t pf_a_bytes, pf_b_bytes;
 };
 
 size_t gemv_smem_bytes(int K, int mr, int unp);
@@ -56,8 +58,6 @@ struct StreamGeom {
     int tiles, tiles_per_cta, grid;
     int smem;           // dynamic shared memory bytes
 };
-// Workspace bytes of the K-split tensor-core GEMV for N rows and reduction length K
-// (0 when that kernel does not apply); counters first, then partial sums.
 // False when the shape or alignment does not fit the streaming kernel.
 bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp);
 int launch_gemv_stream(int pro, int epi, const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl,

@@ -18,6 +18,8 @@
 // up row n (SiLU), and rotate-half partners i, i+64 of one head (RoPE).
 // Every wait is bounded: on a timeout the kernel records I4 device error 1
 // and stops issuing work.
+#include <type_traits>
+
 #include "common.cuh"
 #include "gemv.cuh"
 #include "async.cuh"
@@ -290,6 +292,22 @@ __device__ __forceinline__ void mma_16816_z(float (&d)[4], uint32_t a0, uint32_t
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
+// This CTA's share of an L2 prefetch of [base, base + bytes): 16-byte granules split
+// evenly over the grid.
+__device__ __forceinline__ void prefetch_share(const void *base, size_t bytes) {
+    if (!base || !bytes) return;
+    const size_t granules = bytes >> 4, per = (granules + gridDim.x - 1) / gridDim.x;
+    const size_t g0 = (size_t)blockIdx.x * per;
+    if (g0 >= granules) return;
+    const size_t n = (granules - g0) < per ? (granules - g0) : per;
+    const char *p = reinterpret_cast<const char *>(base) + (g0 << 4);
+    for (size_t done = 0; done < n; done += (1u << 20) >> 4) {  // at most 1 MiB per instruction
+        const size_t m = (n - done) < ((1u << 20) >> 4) ? (n - done) : ((1u << 20) >> 4);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + (done << 4)), "r"((unsigned)(m << 4))
+                     : "memory");
+    }
+}
+
 template <int PRO, class Group>
 __device__ __forceinline__ void stage_x_tc(const GemvArgs &a, uint4 *xt, float *sx8, float *red, const Group &grp) {
     const int nb = tc_blocks(a.K), groups = a.K >> 7;
@@ -360,6 +378,10 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvAr
                     break;
                 }
                 issue_tile<EPI, R>(a, t_begin + i, ring + (size_t)s * geo.stage_bytes, &full[s], pol);
+                if (i == (n_tiles < S ? n_tiles : S) - 1) {  // ring filled: spare DRAM time goes to the next kernel
+                    prefetch_share(a.pf_a, a.pf_a_bytes);
+                    prefetch_share(a.pf_b, a.pf_b_bytes);
+                }
             }
         }
     } else {
@@ -400,12 +422,18 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvAr
                 const unsigned char *wb = st + (size_t)trb * wrow + 16 * lane;
                 const uint16_t *sa = reinterpret_cast<const uint16_t *>(st + (size_t)R * wrow) + tra * groups;
                 const uint16_t *sb = reinterpret_cast<const uint16_t *>(st + (size_t)R * wrow) + trb * groups;
-#pragma unroll 2
-                for (int b = b0; b < b1; ++b) {
-                    // the lane's 32 weights of each row; past K (partial last block) all-zero codes (u = 0)
-                    const bool in = 1024 * b + 32 * lane < K;
-                    uint4 qa = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u), qb = qa;
-                    if (in) {
+                float2 tot = make_float2(0.f, 0.f);  // rows (r, r')
+                // one block: the lane's 32 weights of each row, 8 MMAs, then this lane's group if it holds D[g][g]
+                auto block = [&](int b, auto partial) {
+                    uint4 qa, qb;
+                    if constexpr (decltype(partial)::value) {  // past K: all-zero codes (u = 0)
+                        qa = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+                        qb = qa;
+                        if (1024 * b + 32 * lane < K) {
+                            qa = *reinterpret_cast<const uint4 *>(wa + 512 * b);
+                            qb = *reinterpret_cast<const uint4 *>(wb + 512 * b);
+                        }
+                    } else {
                         qa = *reinterpret_cast<const uint4 *>(wa + 512 * b);
                         qb = *reinterpret_cast<const uint4 *>(wb + 512 * b);
                     }
@@ -426,15 +454,22 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvAr
                         }
                     }
                     const int j = 8 * b + g;  // this lane's group
-                    if (diag && j < groups) {
+                    if (diag && (!decltype(partial)::value || j < groups)) {
                         const bool odd = g & 1;
-                        const float la = odd ? lo[1] : lo[0], ha = odd ? hi[1] : hi[0];
-                        const float lb = odd ? lo[3] : lo[2], hb = odd ? hi[3] : hi[2];
+                        const float2 l2 = odd ? make_float2(lo[1], lo[3]) : make_float2(lo[0], lo[2]);
+                        const float2 h2 = odd ? make_float2(hi[1], hi[3]) : make_float2(hi[0], hi[2]);
                         const float sxj = sx8[j];
-                        tot_a = fmaf(fmaf(ha, 0.0625f, la) * 16777216.0f - sxj, half_bits_to_float(sa[j]), tot_a);
-                        tot_b = fmaf(fmaf(hb, 0.0625f, lb) * 16777216.0f - sxj, half_bits_to_float(sb[j]), tot_b);
+                        const float2 v = ffma2(ffma2(h2, make_float2(0.0625f, 0.0625f), l2),
+                                               make_float2(16777216.0f, 16777216.0f), make_float2(-sxj, -sxj));
+                        tot = ffma2(v, make_float2(half_bits_to_float(sa[j]), half_bits_to_float(sb[j])), tot);
                     }
-                }
+                };
+                const int b_full = b1 < (K >> 10) ? b1 : (K >> 10);
+#pragma unroll 2
+                for (int b = b0; b < b_full; ++b) block(b, std::false_type{});
+                for (int b = b_full > b0 ? b_full : b0; b < b1; ++b) block(b, std::true_type{});
+                tot_a = tot.x;
+                tot_b = tot.y;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
