@@ -160,6 +160,31 @@ __device__ __forceinline__ void st_cluster_f2(uint32_t addr, float a, float b) {
 }
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 
+// oh[h] = sum_k cw[k][h] * part[k][d][h] over n <= N partials laid out [k][dim][head]
+template <int N>
+__device__ __forceinline__ void combine(float (&oh)[kMaxGroup], const float *part, const float (*cw)[kMaxGroup],
+                                        int d, int n = N) {
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) oh[h] = 0.f;
+#pragma unroll
+    for (int k = 0; k < N; ++k) {
+        if (k < n) {
+            const float4 lo = *reinterpret_cast<const float4 *>(part + ((size_t)k * kHeadDim + d) * kMaxGroup);
+            const float4 hi = *reinterpret_cast<const float4 *>(part + ((size_t)k * kHeadDim + d) * kMaxGroup + 4);
+            const float4 wl = *reinterpret_cast<const float4 *>(&cw[k][0]);
+            const float4 wh = *reinterpret_cast<const float4 *>(&cw[k][4]);
+            oh[0] = fmaf(wl.x, lo.x, oh[0]);
+            oh[1] = fmaf(wl.y, lo.y, oh[1]);
+            oh[2] = fmaf(wl.z, lo.z, oh[2]);
+            oh[3] = fmaf(wl.w, lo.w, oh[3]);
+            oh[4] = fmaf(wh.x, hi.x, oh[4]);
+            oh[5] = fmaf(wh.y, hi.y, oh[5]);
+            oh[6] = fmaf(wh.z, hi.z, oh[6]);
+            oh[7] = fmaf(wh.w, hi.w, oh[7]);
+        }
+    }
+}
+
 // weight of a partial with maximum m under the merged maximum M (0 for an empty partial)
 __device__ __forceinline__ float merge_weight(float m, float M) {
     return m == -INFINITY ? 0.f : exp2f(m - (M == -INFINITY ? 0.f : M));
@@ -170,7 +195,7 @@ __device__ __forceinline__ float merge_weight(float m, float M) {
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) paged_gqa_decode_kernel(const AttnParams p) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ float2 wml[kMaxCluster][kMaxGroup];  // (m, l) of the 4 warps, later of the cluster's CTAs
-    __shared__ float cw[kMaxCluster][kMaxGroup];    // merge weights
+    __shared__ __align__(16) float cw[kMaxCluster][kMaxGroup];  // merge weights
     __shared__ float cM[kMaxGroup], cL[kMaxGroup];
     __shared__ int is_last;
 
@@ -352,36 +377,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) paged_gqa_decode_kernel(
         *reinterpret_cast<float2 *>(r + 8 * kMaxGroup) = make_float2(o[im][2], o[im][3]);
     }
     __syncthreads();
-    if (tid < kMaxGroup) {
-        const int h = tid;
-        float M = -INFINITY;
-        for (int k = 0; k < kWarps; ++k) M = fmaxf(M, wml[k][h].x);
-        float L = 0.f;
-        for (int k = 0; k < kWarps; ++k) {
-            const float wt = merge_weight(wml[k][h].x, M);
-            cw[k][h] = wt;
-            L = fmaf(wt, wml[k][h].y, L);
+    if (tid < 32) {  // lane 4 h + k: weight of warp k's partial of head h
+        const int h = tid >> 2, k = tid & 3;
+        const float2 v = wml[k][h];
+        float M = fmaxf(v.x, __shfl_xor_sync(0xffffffffu, v.x, 1));
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
+        const float wt = merge_weight(v.x, M);
+        float L = wt * v.y;
+        L += __shfl_xor_sync(0xffffffffu, L, 1);
+        L += __shfl_xor_sync(0xffffffffu, L, 2);
+        cw[k][h] = wt;
+        if (k == 0) {
+            cM[h] = M;
+            cL[h] = L;
         }
-        cM[h] = M;
-        cL[h] = L;
     }
     __syncthreads();
     float oh[kMaxGroup];
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) oh[h] = 0.f;
-#pragma unroll
-    for (int k = 0; k < kWarps; ++k) {
-        const float4 lo = *reinterpret_cast<const float4 *>(wo + ((size_t)k * kHeadDim + d) * kMaxGroup);
-        const float4 hi = *reinterpret_cast<const float4 *>(wo + ((size_t)k * kHeadDim + d) * kMaxGroup + 4);
-        oh[0] = fmaf(cw[k][0], lo.x, oh[0]);
-        oh[1] = fmaf(cw[k][1], lo.y, oh[1]);
-        oh[2] = fmaf(cw[k][2], lo.z, oh[2]);
-        oh[3] = fmaf(cw[k][3], lo.w, oh[3]);
-        oh[4] = fmaf(cw[k][4], hi.x, oh[4]);
-        oh[5] = fmaf(cw[k][5], hi.y, oh[5]);
-        oh[6] = fmaf(cw[k][6], hi.z, oh[6]);
-        oh[7] = fmaf(cw[k][7], hi.w, oh[7]);
-    }
+    combine<kWarps>(oh, wo, cw, d);
 
     // ---------------- push this CTA's partial into the cluster leader (rank 0)
     cluster_wait();  // every CTA of the cluster has started
@@ -398,39 +411,30 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) paged_gqa_decode_kernel(
     // ---------------- leader: merge the cluster's CTAs
     const float *co = reinterpret_cast<const float *>(gbase + kRecvOff);
     const float2 *cml = reinterpret_cast<const float2 *>(gbase + kRecvMlOff);
-    if (tid < kMaxGroup) {
-        const int h = tid;
-        float M = -INFINITY;
-        for (int k = 0; k < CL; ++k) M = fmaxf(M, cml[k * kMaxGroup + h].x);
-        float L = 0.f;
-        for (int k = 0; k < CL; ++k) {
-            const float wt = merge_weight(cml[k * kMaxGroup + h].x, M);
-            cw[k][h] = wt;
-            L = fmaf(wt, cml[k * kMaxGroup + h].y, L);
+    if (tid < 64) {  // lane 8 h + k: normalised weight of rank k's partial of head h
+        const int h = tid >> 3, k = tid & 7;
+        const float2 v = k < CL ? cml[k * kMaxGroup + h] : make_float2(-INFINITY, 0.f);
+        float M = fmaxf(v.x, __shfl_xor_sync(0xffffffffu, v.x, 1));
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 4));
+        const float wt = merge_weight(v.x, M);
+        float L = wt * v.y;
+        L += __shfl_xor_sync(0xffffffffu, L, 1);
+        L += __shfl_xor_sync(0xffffffffu, L, 2);
+        L += __shfl_xor_sync(0xffffffffu, L, 4);
+        cw[k][h] = wt * (1.0f / L);
+        if (k == 0) {
+            cM[h] = M;
+            cL[h] = L;
         }
-        cM[h] = M;
-        cL[h] = L;
     }
     __syncthreads();
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) oh[h] = 0.f;
-    for (int k = 0; k < CL; ++k) {
-        const float4 lo = *reinterpret_cast<const float4 *>(co + ((size_t)k * kHeadDim + d) * kMaxGroup);
-        const float4 hi = *reinterpret_cast<const float4 *>(co + ((size_t)k * kHeadDim + d) * kMaxGroup + 4);
-        oh[0] = fmaf(cw[k][0], lo.x, oh[0]);
-        oh[1] = fmaf(cw[k][1], lo.y, oh[1]);
-        oh[2] = fmaf(cw[k][2], lo.z, oh[2]);
-        oh[3] = fmaf(cw[k][3], lo.w, oh[3]);
-        oh[4] = fmaf(cw[k][4], hi.x, oh[4]);
-        oh[5] = fmaf(cw[k][5], hi.y, oh[5]);
-        oh[6] = fmaf(cw[k][6], hi.z, oh[6]);
-        oh[7] = fmaf(cw[k][7], hi.w, oh[7]);
-    }
+    combine<kMaxCluster>(oh, co, cw, d, CL);  // the cluster's output, normalised
     uint16_t *out = p.out + ((size_t)b * p.Hq + g * G) * kHeadDim + d;
     if (w.clusters == 1) {
 #pragma unroll
         for (int h = 0; h < kMaxGroup; ++h)
-            if (h < G) out[(size_t)h * kHeadDim] = float_to_half_bits(oh[h] / cL[h]);
+            if (h < G) out[(size_t)h * kHeadDim] = float_to_half_bits(oh[h]);
         return;
     }
 
@@ -467,10 +471,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) paged_gqa_decode_kernel(
 #pragma unroll
         for (int sh = 16; sh > 0; sh >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
         float L = 0.f;
-        for (int k = lane; k < n_cl; k += 32) {
-            const float wt = merge_weight(ch[k], M);
+        for (int k = lane; k < n_cl; k += 32) {  // the partials are normalised: weight 2^(m_k - M) l_k
+            const float wt = merge_weight(ch[k], M) * lh[k];
             ch[k] = wt;
-            L = fmaf(wt, lh[k], L);
+            L += wt;
         }
         L = warp_sum(L);
         const float inv = 1.0f / L;

@@ -482,26 +482,25 @@ __device__ __forceinline__ void epilogue(const GemvArgs &a, int p, int ra, int r
 struct EpiIn {
     float a, b;
     float2 cs;
+    int page;
 };
 
-// Per-CTA constants of EPI_ROPE_KV: the position and its page (read once, after the dependency wait).
+// Per-CTA constant of EPI_ROPE_KV: the position (read once, after the dependency wait; the page-table
+// entry of its page is read with each tile's other epilogue inputs).
 struct EpiCta {
-    int pos, page;
+    int pos;
 };
 
 template <int EPI>
 __device__ __forceinline__ EpiCta epi_cta(const GemvArgs &a) {
-    EpiCta c = {0, 0};
-    if constexpr (EPI == EPI_ROPE_KV) {
-        c.pos = *a.pos;
-        if (c.pos >= 0 && c.pos < a.max_ctx) c.page = a.page_table[c.pos / a.page_size];
-    }
+    EpiCta c = {0};
+    if constexpr (EPI == EPI_ROPE_KV) c.pos = *a.pos;
     return c;
 }
 
 template <int EPI>
 __device__ __forceinline__ EpiIn epi_load(const GemvArgs &a, int p, int ra, int rb, const EpiCta &c) {
-    EpiIn e = {0.f, 0.f, make_float2(0.f, 0.f)};
+    EpiIn e = {0.f, 0.f, make_float2(0.f, 0.f), 0};
     if constexpr (EPI == EPI_RESID) {
         const uint16_t *r = reinterpret_cast<const uint16_t *>(a.y);
         e.a = half_bits_to_float(r[ra]);
@@ -509,7 +508,10 @@ __device__ __forceinline__ EpiIn epi_load(const GemvArgs &a, int p, int ra, int 
     } else if constexpr (EPI == EPI_ROPE_KV) {
         e.a = half_bits_to_float(a.bias[ra]);
         e.b = half_bits_to_float(a.bias[rb]);
-        if (c.pos >= 0 && c.pos < a.max_ctx && (p >> 6) < a.n_q + a.n_kv) e.cs = a.rope_cs[(size_t)c.pos * 64 + (p & 63)];
+        if (c.pos >= 0 && c.pos < a.max_ctx) {
+            if ((p >> 6) < a.n_q + a.n_kv) e.cs = a.rope_cs[(size_t)c.pos * 64 + (p & 63)];
+            if ((p >> 6) >= a.n_q) e.page = a.page_table[c.pos / a.page_size];
+        }
     } else if constexpr (EPI == EPI_F16 || EPI == EPI_F32) {
         if (a.bias) {
             e.a = half_bits_to_float(a.bias[ra]);
@@ -559,13 +561,13 @@ __device__ __forceinline__ void epilogue_in(const GemvArgs &a, int p, int ra, in
                 a.q_out[head * 128 + i + 64] = ob;
             } else {
                 const int g = head - a.n_q;
-                const size_t off = (((size_t)c.page * a.n_kv + g) * a.page_size + c.pos % a.page_size) * 128;
+                const size_t off = (((size_t)e.page * a.n_kv + g) * a.page_size + c.pos % a.page_size) * 128;
                 a.k_pool[off + i] = oa;
                 a.k_pool[off + i + 64] = ob;
             }
         } else {
             const int g = head - a.n_q - a.n_kv;
-            const size_t off = (((size_t)c.page * a.n_kv + g) * a.page_size + c.pos % a.page_size) * 128;
+            const size_t off = (((size_t)e.page * a.n_kv + g) * a.page_size + c.pos % a.page_size) * 128;
             a.v_pool[off + i] = float_to_half_bits(xa);
             a.v_pool[off + i + 64] = float_to_half_bits(xb);
         }

@@ -388,6 +388,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvAr
         // ---------------- consumers
         const NamedGroup<32, kConsumers> grp;
         grid_dep_wait();
+        const EpiCta ecta = epi_cta<EPI>(a);  // issued before the staging so its latency overlaps it
         stage_x_tc<PRO>(a, xt, sx8, red, grp);
         grp.sync();
         grid_dep_launch();
@@ -397,7 +398,6 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvAr
         const int pr = warp / WP, wp = warp % WP;
         const int b0 = (wp * nb) / WP, b1 = ((wp + 1) * nb) / WP;
         const int tra = kPaired<EPI> ? pr : 2 * pr, trb = kPaired<EPI> ? pr + PP : 2 * pr + 1;
-        const EpiCta ecta = epi_cta<EPI>(a);
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
             const int s = i % S, n = i / S, t = t_begin + i;
@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvAr
             int pa, pb;
             pair_rows<EPI>(a, p, pa, pb);
             const bool epi_lane = lane == 0 && wp == 0 && trb < na + nb_rows;
-            EpiIn ein = {0.f, 0.f, make_float2(0.f, 0.f)};
+            EpiIn ein = {0.f, 0.f, make_float2(0.f, 0.f), 0};
             if (epi_lane) ein = epi_load<EPI>(a, p, pa, pb, ecta);
             if (ok && !mbar_wait(&full[s], (unsigned)(n & 1))) {
                 record_error(&g_device_error, 1);
