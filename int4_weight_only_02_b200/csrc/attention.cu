@@ -202,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) paged_gqa_decode_kernel(
     const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = p.Hq / p.Hkv, P = p.page_size, CL = p.cluster;
+    const int pshift = __ffs(P) - 1;  // page_size is a power of two: t / P == t >> pshift
     const int max_ctx = p.max_pages * P;
     int ctx = p.ctx_len[b];  // advanced by an earlier step's last kernel, never by this kernel's predecessor
     ctx = ctx < 1 ? 1 : (ctx > max_ctx ? max_ctx : ctx);
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) paged_gqa_decode_kernel(
     const uint32_t ring = base + warp * kStages * kWarpStageBytes;  // this warp's stages
 
     // ---------------- staging: lane copies 16-byte chunk (lane & 15) of rows (lane >> 4) + 2j, j < 8
-    const int last_page = (ctx - 1) / P;
+    const int last_page = (ctx - 1) >> pshift;
     const int32_t *table = p.page_table + (size_t)b * p.max_pages;
     const size_t head_rows = (size_t)g * P;  // row offset of kv head g inside a page
     auto slab = [&](int i) { return (tile0 + i) * kTileTokens + warp * kWarpTokens; };  // first token of tile i
@@ -231,8 +232,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) paged_gqa_decode_kernel(
         ea = eb = 0;
         if (i < n_my && t < ctx) {
             const int tl = t + kWarpTokens - 1 < ctx ? t + kWarpTokens - 1 : ctx - 1;
-            ea = table[t / P];
-            eb = table[tl / P];
+            ea = table[t >> pshift];
+            eb = table[tl >> pshift];
         }
     };
     int cur_batch = 0, ca, cb, na, nb;
@@ -252,22 +253,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) paged_gqa_decode_kernel(
         const int t = slab(i);
         if (!waited && t < ctx) {
             const int tl = t + kWarpTokens - 1 < ctx ? t + kWarpTokens - 1 : ctx - 1;
-            if (tl / P == last_page) {
+            if ((tl >> pshift) == last_page) {
                 grid_dep_wait();  // the current page's new row comes from the preceding kernel
                 waited = true;
             }
         }
         const uint32_t st = ring + (i % kStages) * kWarpStageBytes + chunk_off;
-        const int pa = t / P;
+        const int pa = t >> pshift;
+        // element offsets of this kv head's rows in the two pages the warp's 16 tokens can touch
+        const size_t base_a = (((size_t)ea * p.Hkv) * P + head_rows) * kHeadDim + chunk * 8;
+        const size_t base_b = (((size_t)eb * p.Hkv) * P + head_rows) * kHeadDim + chunk * 8;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int r = row_lo + 2 * j, tok = t + r;
             if (tok < ctx) {
-                const int e = tok / P == pa ? ea : eb;
-                const size_t row = ((size_t)e * p.Hkv) * P + head_rows + (tok % P);
+                const size_t off = ((tok >> pshift) == pa ? base_a : base_b) + (size_t)(tok & (P - 1)) * kHeadDim;
                 const uint32_t dst = st + r * 128 + (((chunk & 7) ^ (r & 7)) << 4);
-                cp_async16(dst, p.k_pool + row * kHeadDim + chunk * 8);
-                cp_async16(dst + 2 * kRegionBytes, p.v_pool + row * kHeadDim + chunk * 8);
+                cp_async16(dst, p.k_pool + off);
+                cp_async16(dst + 2 * kRegionBytes, p.v_pool + off);
             }
         }
     };
