@@ -503,6 +503,10 @@ def main():
     o_bytes = h * (h // 2) + h * (h // 128) * 2 + h * 2 + 2 * h * 2
     o_ms = time_kernel(lambda li: 5 * li + 2)
     attn_ms = time_kernel(lambda li: 5 * li + 1)
+    # lm_head: the last kernel of the step, launched 28 times (it also advances the sequence state,
+    # which nothing reads afterwards)
+    lm_bytes = shape.vocab * (h // 2) + shape.vocab * (h // 128) * 2 + shape.vocab * 4 + 2 * h * 2
+    lm_ms = time_kernel(lambda li: n_k - 1)
     torch.cuda.synchronize()
     # restore a consistent residual/KV state is not needed afterwards: nothing else runs
 
@@ -535,7 +539,8 @@ def main():
             "gate_up": {"us": round(gu_ms * 1e3, 2), "GBs": round(gu_gbs, 1)},
             "down": {"us": round(down_ms * 1e3, 2), "GBs": round(down_bytes / (down_ms * 1e-3) / 1e9, 1)},
             "attention": {"us": round(attn_ms * 1e3, 2),
-                          "GBs": round(2 * shape.n_kv * shape.head_dim * 2 * (ctx1 - 1) / (attn_ms * 1e-3) / 1e9, 1)}},
+                          "GBs": round(2 * shape.n_kv * shape.head_dim * 2 * (ctx1 - 1) / (attn_ms * 1e-3) / 1e9, 1)},
+            "lm_head": {"us": round(lm_ms * 1e3, 2), "GBs": round(lm_bytes / (lm_ms * 1e-3) / 1e9, 1)}},
         "step_roofline": {"bytes_per_step": int(step_bytes), "achieved_GBs": round(step_gbs, 1),
                           "frac_of_8TBs": round(step_gbs / NOMINAL_HBM_GBS, 4),
                           "frac_of_measured": round(step_gbs / peak, 4)},
