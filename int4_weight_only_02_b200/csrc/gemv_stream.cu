@@ -7,17 +7,20 @@
 // To Build Your Own LLM Runtime From Scratch": INT4 dequantisation fused into
 // the decode GEMVs). Issuing loads from the consumer registers serialises
 // load and compute inside each warp; here the bytes in flight per SM are the
-// ring (up to ~190 KB), independent of the compute. The producer issues its
-// first copies before the kernel waits on its predecessor (programmatic
-// dependent launch), so the weight stream of kernel N+1 starts while kernel N
-// drains. One CTA per SM, tiles of whole rows assigned in contiguous ranges.
+// two CTAs' rings (~90-100 KB each), independent of the compute. The producer
+// issues its first copies before the kernel waits on its predecessor
+// (programmatic dependent launch), so the weight stream of kernel N+1 can start
+// while kernel N drains. Two CTAs per SM, tiles of whole rows assigned in
+// balanced contiguous ranges.
 //
-// Tiles: R = 16 rows (K <= 4096; a warp per row pair, x in registers) or R =
-// 2 rows (larger K; all consumer threads split K, x from shared memory). Row-pair epilogues keep both rows of a pair
-// in one tile: consecutive rows (plain / residual / logits), gate row n with
-// up row n (SiLU), and rotate-half partners i, i+64 of one head (RoPE).
-// Every wait is bounded: on a timeout the kernel records I4 device error 1
-// and stops issuing work.
+// Tiles: R = 16 rows (K <= 4096) or R = 2 rows (larger K). Row-pair epilogues
+// keep both rows of a pair in one tile: consecutive rows (plain / residual /
+// logits), gate row n with up row n (SiLU), and rotate-half partners i, i+64 of
+// one head (RoPE). Two consumers share the producer and the tiles: the CUDA-core
+// one (gemv_stream_kernel: a warp per row pair with x in registers for R = 16,
+// all consumer threads splitting K with x in shared memory for R = 2) and the
+// tensor-core one (gemv_tc_kernel, below). Every wait is bounded: on a timeout
+// the kernel records I4 device error 1 and stops issuing work.
 #include <type_traits>
 
 #include "common.cuh"
