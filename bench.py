@@ -340,6 +340,61 @@ def run_attention_sweep(args):
     return 0
 
 
+def run_gemv_batch(args):
+    """INT4 GEMV at the gate/up shape (K = 3584, N = 37888, plain fp16 output) for M = 1, 2, 4, 8 vectors:
+    the first step of batched decode. Each launch is L2-cold (a graph of (flush, GEMV) pairs minus the
+    flushes); one JSON line per M with weight GB/s against the measured HBM peak."""
+    import numpy as np
+    import torch
+
+    import int4_weight_only_02_b200 as i4
+    from int4_weight_only_02_b200 import synth
+    dev = torch.device("cuda", 0)
+    peak, peak_kind = measured_peaks()
+    n, k = 37888, 3584
+    w, s, _, _ = synth.gemv_case(n, k, seed=0)
+    wd, sd = torch.from_numpy(w).to(dev), torch.from_numpy(s).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    reps = 10
+    for m in (1, 2, 4, 8):
+        x = torch.randn((m, k), generator=torch.Generator(device=dev).manual_seed(m), device=dev).half()
+        y = torch.empty((m, n), dtype=torch.float16, device=dev)
+
+        def graph_ms(with_gemv):
+            side = torch.cuda.Stream()
+            g = torch.cuda.CUDAGraph()
+            torch.cuda.synchronize()
+            with torch.cuda.stream(side):
+                i4.int4_gemv(wd, sd, x, y=y, stream=side)
+                with torch.cuda.graph(g, stream=side):
+                    for _ in range(reps):
+                        flush.add_(1)
+                        if with_gemv:
+                            i4.int4_gemv(wd, sd, x, y=y, stream=side)
+            torch.cuda.synchronize()
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            best = None
+            for _ in range(3):
+                e0.record()
+                g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                t = e0.elapsed_time(e1) / reps
+                best = t if best is None else min(best, t)
+            return best
+
+        ms = graph_ms(True) - graph_ms(False)
+        wbytes = n * (k // 2) + n * (k // 128) * 2
+        gbs = wbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({"gemv_batch": m, "N": n, "K": k, "us": round(ms * 1e3, 2), "weight_GBs": round(gbs, 1),
+                          "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
+                          "vector_GEMVs_per_s": round(m / (ms * 1e-3), 1), "device_error": i4.device_error()}),
+              flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -361,6 +416,8 @@ def main():
     ap.add_argument("--attention-sweep", action="store_true",
                     help="paged attention sweep over contexts, page sizes 16/64 and batches 1/8/32 (KV GB/s)")
     ap.add_argument("--sweep-contexts", default="512,2048,8192,32768")
+    ap.add_argument("--gemv-batch", action="store_true",
+                    help="INT4 GEMV at the gate/up shape for 1, 2, 4 and 8 vectors (weight GB/s)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -368,6 +425,8 @@ def main():
         return run_profile_kernel(args)
     if args.attention_sweep:
         return run_attention_sweep(args)
+    if args.gemv_batch:
+        return run_gemv_batch(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 

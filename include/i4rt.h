@@ -268,8 +268,9 @@ I4_API int decode_step_launch_kernel(i4_graph *g, int index, void *stream);
  *            values, 1 offset-binary fp16 subnormals with a sum(x) correction
  *            (both fp16 x fp16 -> fp32 FMAs), 2 fp32 values from an exponent
  *            trick (packed fp32 FMAs), 3 the subnormal fields as the A operand of
- *            mma.sync (tensor cores, fp32 accumulate), 4 (default) per launch: 3
- *            for a single vector (M == 1), else 0;
+ *            mma.sync (tensor cores, fp32 accumulate; for M = 2..8 the vectors are
+ *            the MMA's N columns, rows of up to 4096 weights), 4 (default): 3
+ *            where it applies, else 0;
  *   "stream" 0/1: use the bulk-copy pipelined GEMV where the shape allows it
  *            (M == 1, K % 512 == 0, 16-byte aligned w and scales), default 1;
  *   "stream_smem_kb" 32..227: shared memory budget of that kernel's ring;

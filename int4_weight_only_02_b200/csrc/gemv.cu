@@ -174,7 +174,7 @@ int g_default_unpack = UNPACK_AUTO;
 
 int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool pdl, int unp, int max_ctas) {
     if (unp < 0) unp = g_default_unpack;
-    if (unp == UNPACK_AUTO) unp = a.M == 1 ? UNPACK_MMA : UNPACK_EXACT;
+    if (unp == UNPACK_AUTO) unp = a.M <= 8 ? UNPACK_MMA : UNPACK_EXACT;
     StreamGeom geo;
     if (max_ctas == 0 && stream_geometry(epi, a, geo, unp)) return launch_gemv_stream(pro, epi, a, geo, stream, pdl, unp);
     if (max_ctas == 0 && unp == UNPACK_MMA && stream_geometry(epi, a, geo, UNPACK_SUBNORMAL))

@@ -507,6 +507,162 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvAr
     if constexpr (EPI == EPI_ARGMAX) finish_step(a, best);
 }
 
+// ---------------------------------------------------------------- batched tensor-core consumer (M = 2..8)
+//
+// y[m][n] = x[m] . w[n] for up to 8 vectors (a batch of decode steps): the 8 B
+// columns of mma.m16n8k16 are the 8 vectors, the 16 A rows are 16 weight rows
+// of a tile, so every D entry is useful and each unpacked weight serves the whole
+// batch. Lane (g, c) reads 16 bytes (32 weights) of rows g and g + 8 per group of
+// 128 weights; its B fragment is vector g's x at the same k (staged once per CTA
+// in lane order; vectors past M are zero). The 8 consumer warps split the tile's
+// groups and their partial sums meet in shared memory. Rows only up to 4096
+// weights (the 8 staged vectors take 2 bytes x 8 x K of shared memory), one CTA
+// per SM.
+constexpr int kTcbBudget = 212 * 1024;  // + 8 KB of static partial sums within the 227 KB per CTA
+
+__host__ __device__ constexpr long long tcb_x_bytes(int K) { return (long long)(K / 128) * 2048 + 8LL * (K / 128) * 4; }
+
+template <class Group>
+__device__ __forceinline__ void stage_x_tcb(const GemvArgs &a, uint4 *xb, float *sx8, const Group &grp) {
+    const int groups = a.K >> 7, nwords = a.K >> 3;
+    for (int i = grp.tid(); i < 8 * nwords; i += grp.size()) {  // i = vector * nwords + word
+        const int n = i / nwords, wd = i % nwords;
+        const int j = wd >> 4, c = (wd >> 2) & 3, w = wd & 3;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (n < a.M) {
+            const uint4 pp = permute_pairs(*reinterpret_cast<const uint4 *>(a.x + (size_t)n * a.K + 8 * wd));
+            v = make_uint4(pp.x, pp.z, pp.y, pp.w);  // (x0,x4) (x2,x6) | (x1,x5) (x3,x7)
+        }
+        xb[(j * 4 + w) * 32 + 4 * n + c] = v;
+    }
+    grp.sync();
+    for (int i = grp.tid(); i < 8 * groups; i += grp.size()) {  // i = vector * groups + group
+        const int n = i / groups, j = i % groups;
+        float t = 0.f;
+        for (int w = 0; w < 4; ++w)
+            for (int c = 0; c < 4; ++c) {
+                const uint4 e = xb[(j * 4 + w) * 32 + 4 * n + c];
+                const uint32_t v[4] = {e.x, e.y, e.z, e.w};
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&v[q]));
+                    t += f.x + f.y;
+                }
+            }
+        sx8[n * groups + j] = 8.0f * t;
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kStreamThreads, 1) gemv_tcb_kernel(const GemvArgs a, const StreamGeom geo) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full[kMaxStages];
+    __shared__ __align__(8) uint64_t empty[kMaxStages];
+    __shared__ float red[2][kConsumerWarps][16][8];  // per-warp partial sums [row][vector], tile parity
+
+    const int K = a.K, wrow = K >> 1, groups = K >> 7;
+    const int S = geo.stages;
+    unsigned char *ring = smem;
+    uint4 *xb = reinterpret_cast<uint4 *>(smem + (size_t)S * geo.stage_bytes);
+    float *sx8 = reinterpret_cast<float *>(xb + (size_t)groups * 128);
+    const int t_begin = (int)(((long long)blockIdx.x * geo.tiles) / gridDim.x);
+    const int t_end = (int)(((long long)(blockIdx.x + 1) * geo.tiles) / gridDim.x);
+    const int n_tiles = t_end - t_begin;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (threadIdx.x < 32) {
+        if (threadIdx.x == 0) {
+            const uint64_t pol = evict_first_policy();
+            for (int i = 0; i < n_tiles; ++i) {
+                const int s = i % S, n = i / S;
+                if (n > 0 && !mbar_wait(&empty[s], (unsigned)((n - 1) & 1))) {
+                    record_error(&g_device_error, 1);
+                    break;
+                }
+                issue_tile<EPI, 16>(a, t_begin + i, ring + (size_t)s * geo.stage_bytes, &full[s], pol);
+            }
+        }
+        return;
+    }
+    const NamedGroup<32, kConsumers> grp;
+    grid_dep_wait();
+    stage_x_tcb(a, xb, sx8, grp);
+    grp.sync();
+    grid_dep_launch();
+    const int c_id = grp.tid(), warp = c_id >> 5, lane = c_id & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int j0 = (warp * groups) / kConsumerWarps, j1 = ((warp + 1) * groups) / kConsumerWarps;
+    bool ok = true;
+    for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % S, n = i / S, t = t_begin + i;
+        if (ok && !mbar_wait(&full[s], (unsigned)(n & 1))) {
+            record_error(&g_device_error, 1);
+            ok = false;
+        }
+        const int r0 = t * 16, rows = (a.N - r0) < 16 ? (a.N - r0) : 16;
+        float tot[4] = {0.f, 0.f, 0.f, 0.f};  // (row g, vec 2c) (row g, vec 2c+1) (row g+8, vec 2c) (row g+8, vec 2c+1)
+        if (ok) {
+            const unsigned char *st = ring + (size_t)s * geo.stage_bytes;
+            // rows past the tile's end hold stale bytes: their results are never stored
+            const unsigned char *wg = st + (size_t)g * wrow + 16 * c;
+            const unsigned char *wg8 = st + (size_t)(g + 8) * wrow + 16 * c;
+            const uint16_t *sc = reinterpret_cast<const uint16_t *>(st + (size_t)16 * wrow);
+            for (int j = j0; j < j1; ++j) {
+                const uint4 qa = *reinterpret_cast<const uint4 *>(wg + 64 * j);
+                const uint4 qb = *reinterpret_cast<const uint4 *>(wg8 + 64 * j);
+                const uint32_t wra[4] = {qa.x, qa.y, qa.z, qa.w}, wrb[4] = {qb.x, qb.y, qb.z, qb.w};
+                float lo[4], hi[4];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const uint4 xc = xb[(j * 4 + w) * 32 + lane];
+                    uint32_t ua[4], ub[4];
+                    unpack_word_subnormal(wra[w], ua);
+                    unpack_word_subnormal(wrb[w], ub);
+                    if (w == 0) {
+                        mma_16816_z(lo, ua[0], ub[0], ua[2], ub[2], xc.x, xc.y);
+                        mma_16816_z(hi, ua[1], ub[1], ua[3], ub[3], xc.z, xc.w);
+                    } else {
+                        mma_16816(lo, ua[0], ub[0], ua[2], ub[2], xc.x, xc.y);
+                        mma_16816(hi, ua[1], ub[1], ua[3], ub[3], xc.z, xc.w);
+                    }
+                }
+                const float sg = half_bits_to_float(sc[g * groups + j]), sg8 = half_bits_to_float(sc[(g + 8) * groups + j]);
+                const float sxa = sx8[(2 * c) * groups + j], sxb = sx8[(2 * c + 1) * groups + j];
+                tot[0] = fmaf(fmaf(hi[0], 0.0625f, lo[0]) * 16777216.0f - sxa, sg, tot[0]);
+                tot[1] = fmaf(fmaf(hi[1], 0.0625f, lo[1]) * 16777216.0f - sxb, sg, tot[1]);
+                tot[2] = fmaf(fmaf(hi[2], 0.0625f, lo[2]) * 16777216.0f - sxa, sg8, tot[2]);
+                tot[3] = fmaf(fmaf(hi[3], 0.0625f, lo[3]) * 16777216.0f - sxb, sg8, tot[3]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        red[i & 1][warp][g][2 * c] = tot[0];
+        red[i & 1][warp][g][2 * c + 1] = tot[1];
+        red[i & 1][warp][g + 8][2 * c] = tot[2];
+        red[i & 1][warp][g + 8][2 * c + 1] = tot[3];
+        grp.sync();
+        if (c_id < 128 && ok) {
+            const int row = c_id >> 3, m = c_id & 7;
+            if (row < rows && m < a.M) {
+                float v = 0.f;
+                for (int w = 0; w < kConsumerWarps; ++w) v += red[i & 1][w][row][m];
+                if (a.bias) v += half_bits_to_float(a.bias[r0 + row]);
+                if constexpr (EPI == EPI_F32)
+                    reinterpret_cast<float *>(a.y)[(size_t)m * a.N + r0 + row] = v;
+                else
+                    reinterpret_cast<uint16_t *>(a.y)[(size_t)m * a.N + r0 + row] = float_to_half_bits(v);
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
 static bool g_stream_enabled = true;
@@ -521,7 +677,26 @@ void set_stream_options(int enabled, int smem_kb) {
 void set_stream_ctas_per_sm(int n) { g_stream_ctas_per_sm = n; }
 
 bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp) {
-    if (!g_stream_enabled || a.M != 1 || a.K % 512 != 0 || a.K > 32768 || a.N < 2) return false;
+    if (!g_stream_enabled || a.K % 512 != 0 || a.K > 32768 || a.N < 2) return false;
+    if (unp == UNPACK_MMA && a.M > 1) {
+        // batched tensor-core kernel: plain x, fp16/fp32 output, rows of up to 4096 weights
+        if (a.M > 8 || !(epi == EPI_F16 || epi == EPI_F32) || a.K > 4096) return false;
+        if (!aligned(a.w, 16) || !aligned(a.s, 16) || !aligned(a.x, 16)) return false;
+        const long long wrow = a.K / 2, srow = a.K / 64;
+        g.R = 16;
+        g.stage_bytes = (int)(((16 * (wrow + srow)) + 127) / 128 * 128);
+        const long long xs_bytes = (tcb_x_bytes(a.K) + 127) / 128 * 128;
+        int stages = (int)((kTcbBudget - xs_bytes) / g.stage_bytes);
+        if (stages > kMaxStages) stages = kMaxStages;
+        if (stages < 2) return false;
+        g.stages = stages;
+        g.tiles = (a.N + 15) / 16;
+        g.grid = g.tiles < kNumSMs ? g.tiles : kNumSMs;
+        g.tiles_per_cta = (g.tiles + g.grid - 1) / g.grid;
+        g.smem = (int)(stages * (long long)g.stage_bytes + xs_bytes);
+        return true;
+    }
+    if (a.M != 1) return false;
     if (unp == UNPACK_MMA) {
         const bool paired = (epi == EPI_SILU || epi == EPI_ROPE_KV);
         const int R = a.K <= 32 * kMaxHalvesPerLane * 16 ? 16 : 2;
@@ -606,8 +781,29 @@ static int launch_tc_t(const GemvArgs &a, const StreamGeom &geo, cudaStream_t st
                       "tensor-core gemv launch");
 }
 
+template <int EPI>
+static int launch_tcb_t(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
+    auto kern = gemv_tcb_kernel<EPI>;
+    static int configured = -1;
+    if (geo.smem > configured) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, geo.smem);
+        if (e != cudaSuccess) return cuda_check(e, "batched tensor-core gemv smem attribute");
+        configured = geo.smem;
+    }
+    if (g_dry_run) return I4_OK;
+    return cuda_check(launch(kern, dim3(geo.grid), dim3(kStreamThreads), (size_t)geo.smem, stream, pdl, a, geo),
+                      "batched tensor-core gemv launch");
+}
+
 template <int PRO, int EPI>
 static int launch_mma_t(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
+    if (a.M > 1) {
+        if constexpr (PRO == PRO_PLAIN && (EPI == EPI_F16 || EPI == EPI_F32)) {
+            return launch_tcb_t<EPI>(a, geo, stream, pdl);
+        } else {
+            return fail(I4_EUNSUPPORTED, "batched tensor-core gemv: plain prologue and fp16/fp32 output only");
+        }
+    }
     if (geo.R == 16) return launch_tc_t<PRO, EPI, 16>(a, geo, stream, pdl);
     if constexpr (EPI == EPI_SILU || EPI == EPI_ROPE_KV) {
         return fail(I4_EUNSUPPORTED, "tensor-core gemv: paired epilogue needs 16-row tiles");

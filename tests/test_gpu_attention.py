@@ -1,8 +1,9 @@
 """Paged GQA decode attention through the C ABI vs the CPU oracle (needs a B200).
 
 Covers the page-tail lengths (1, P-1, P, P+1, 511, 513), ragged batches over a
-shared permuted page pool (page sizes 16 and 64), long contexts, bit-exact
-page indexing, and bit-identical results under any page permutation.
+shared permuted page pool (page sizes 16 and 64), long contexts, the sweep's
+largest shapes (sampled), bit-exact page indexing, and bit-identical results
+under any page permutation.
 """
 import numpy as np
 import pytest
@@ -51,6 +52,21 @@ def test_ragged_batches(i4lib, cuda, page_size, length, batch):
 @pytest.mark.parametrize("ctx,page_size", [(8192, 16), (32768, 64)])
 def test_long_context(i4lib, cuda, ctx, page_size):
     check_case(i4lib, cuda, [ctx], page_size, seed=11)
+
+
+@pytest.mark.parametrize("length,batch,page_size", [(32768, 8, 16), (8192, 32, 64)])
+def test_sweep_full_size_sampled(i4lib, cuda, length, batch, page_size):
+    """The attention sweep's largest shapes (ragged lengths in [L/2, L], one shared permuted pool) in the
+    launch configuration the sweep times; the oracle checks the longest, the shortest and one more
+    sequence in full."""
+    lens = synth.ragged_lengths(length, batch, seed=length + batch)
+    q, kp, vp, table, ctx = synth.attention_case(lens, page_size=page_size, seed=page_size + batch + 1)
+    got = run_attention(i4lib, cuda, q, kp, vp, table, ctx)
+    for b in sorted({int(np.argmax(ctx)), int(np.argmin(ctx)), batch // 2}):
+        ref = oracle.f16(oracle.paged_attention(q[b], kp, vp, table[b], int(ctx[b])))
+        err = normwise_err(got[b], ref)
+        assert err <= TOL, (b, int(ctx[b]), err)
+    assert np.all(np.isfinite(got.astype(np.float32)))
 
 
 def test_group_sizes(i4lib, cuda):

@@ -132,3 +132,33 @@ def test_tensor_core_kernel_block_edges(i4lib, cuda, n, k):
     torch.cuda.synchronize()
     assert normwise_err(got.cpu().numpy()[0], ref) <= TOL
     assert i4lib.device_error() == 0
+
+
+@pytest.mark.parametrize("n,k,m", [(4608, 3584, 2), (1000, 3584, 4), (3584, 2048, 8), (18, 512, 7)])
+def test_batched_tensor_core_kernel(i4lib, cuda, n, k, m):
+    """M = 2..8 vectors as the MMA's N columns (default path and explicit variant 3): qkv-sized and
+    ragged row counts, fp16 and fp32 outputs, bias."""
+    w, s, x, b = synth.gemv_case(n, k, m=m, seed=10, bias=True)
+    ref = oracle.int4_gemv(w, s, x, b)
+    for unpack in (3, None):
+        got = run_gemv(i4lib, cuda, w, s, x, b, unpack=unpack)
+        assert got.shape == (m, n)
+        assert normwise_err(got, ref) <= TOL, unpack
+    ref32 = oracle.int4_linear(w, s, x, b)
+    got32 = run_gemv(i4lib, cuda, w, s, x, b, out_fp32=True, unpack=3)
+    assert normwise_err(got32, ref32) <= 1e-5
+    assert i4lib.device_error() == 0
+
+
+def test_batched_tensor_core_exact_arithmetic(i4lib, cuda):
+    """Power-of-two scales and small integer x: every vector of the batch comes out bit-exact."""
+    rng = np.random.default_rng(5)
+    n, k, m = 80, 1024, 6
+    q = rng.integers(-8, 8, size=(n, k))
+    s = np.ldexp(1.0, rng.integers(-8, -4, size=(n, k // 128))).astype(np.float16)
+    x = rng.integers(-3, 4, size=(m, k)).astype(np.float16)
+    w = pack_fields(q)
+    got = run_gemv(i4lib, cuda, w, s, x, unpack=3)
+    for i in range(m):
+        ref = oracle.int4_gemv(w, s, x[i], None)
+        assert np.array_equal(got[i].view(np.uint16), ref.view(np.uint16)), i
