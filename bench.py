@@ -395,6 +395,49 @@ def run_gemv_batch(args):
     return 0
 
 
+def run_batched_decode(args):
+    """B sequences of the 7B-shape decoder decoded together (one CUDA graph of library calls per step),
+    each with its own 512-token prompt (teacher-forced, untimed) and page-table row; then K timed steps.
+    One JSON line: tokens/s over all sequences."""
+    import numpy as np
+    import torch
+
+    import int4_weight_only_02_b200 as i4
+    from int4_weight_only_02_b200 import synth
+    dev = torch.device("cuda", 0)
+    B = args.batched_decode
+    shape = synth.QWEN7B
+    model = i4.DeviceModel.synthetic(shape, device=dev)
+    tables = synth.rng_for(0, 9, B).permutation(B * shape.max_pages).astype(np.int32).reshape(B, shape.max_pages)
+    bd = i4.BatchedDecode(model, tables, num_pages=B * shape.max_pages)
+    prompts = np.stack([synth.prompt_tokens(shape, args.prompt, seed=b) for b in range(B)])
+    bd.reset(prompts[:, 0])
+    stream = torch.cuda.current_stream()
+    for t in range(args.prompt):
+        bd.step(stream=stream)
+        if t + 1 < args.prompt:
+            bd.tokens.copy_(torch.from_numpy(prompts[:, t + 1]).to(dev, non_blocking=False))
+    torch.cuda.synchronize()
+    bd.capture()
+    for _ in range(args.warmup):
+        bd.replay()
+    torch.cuda.synchronize()
+    ctx0 = int(bd.ctx_len[0].item())
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        bd.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"batched_decode": B, "metric": "decode tok/s, batch of sequences (7B-shape INT4)",
+                      "value": round(B / (ms * 1e-3), 1), "unit": "tok/s", "ms_per_step": round(ms, 4),
+                      "steps": args.steps, "warmup": args.warmup, "ctx_first": ctx0,
+                      "ctx_last": int(bd.ctx_len[0].item()) - 1, "launches_per_step": (8 + -(-B // bd.down_rows)) * shape.layers + 4,
+                      "device_error": i4.device_error()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -416,6 +459,8 @@ def main():
     ap.add_argument("--attention-sweep", action="store_true",
                     help="paged attention sweep over contexts, page sizes 16/64 and batches 1/8/32 (KV GB/s)")
     ap.add_argument("--sweep-contexts", default="512,2048,8192,32768")
+    ap.add_argument("--batched-decode", type=int, default=0,
+                    help="decode this many sequences together (1..8) through the batched library calls")
     ap.add_argument("--gemv-batch", action="store_true",
                     help="INT4 GEMV at the gate/up shape for 1, 2, 4 and 8 vectors (weight GB/s)")
     args = ap.parse_args()
@@ -427,6 +472,8 @@ def main():
         return run_attention_sweep(args)
     if args.gemv_batch:
         return run_gemv_batch(args)
+    if args.batched_decode:
+        return run_batched_decode(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 

@@ -125,6 +125,17 @@ I4_API int paged_gqa_decode_static(const uint16_t *q, const uint16_t *k_pool, co
                                    int Hkv, int D, int page_size, int max_pages_per_seq, float scale, void *stream);
 
 /*
+ * paged_gqa_decode with the q rows of consecutive sequences q_stride elements
+ * apart (q_stride >= Hq * D, a multiple of 8), so q can be read where a fused
+ * qkv projection left it: q of sequence b is q[b * q_stride .. + Hq * D).
+ * Same workspace, layouts, results and errors as paged_gqa_decode otherwise.
+ */
+I4_API int i4_paged_gqa_decode_strided(const uint16_t *q, long long q_stride, const uint16_t *k_pool,
+                                       const uint16_t *v_pool, const int32_t *page_table, const int32_t *ctx_len,
+                                       uint16_t *out, int B, int Hq, int Hkv, int D, int page_size,
+                                       int max_pages_per_seq, float scale, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Test export: out[b][g][t][:] = pool row of token t (t < ctx_len[b]) for kv
  * head g, in token order (bit-exact page-indexing check). Rows t >= ctx_len[b]
  * are left untouched.  out [B][Hkv][max_ctx][D] fp16.
@@ -179,6 +190,23 @@ I4_API int i4_rope_kv_append(uint16_t *qkv, const int32_t *pos, int B, int Hq, i
  * silu(g) = g / (1 + exp(-g)) in fp32.  gate_up [M][2I] fp16; out [M][I] fp16.
  */
 I4_API int silu_mul(const uint16_t *gate_up, uint16_t *out, int M, int I, void *stream);
+
+/*
+ * Embedding rows of a batch of tokens: out[b][:] = table[t][:] with
+ * t = tokens[b] clamped to [0, vocab). table [vocab][H] fp16, tokens [B] int32
+ * device array, out [B][H] fp16; H % 8 == 0, table and out 16-byte aligned.
+ */
+I4_API int i4_embed_gather(const uint16_t *table, const int32_t *tokens, uint16_t *out, int B, int H, int vocab,
+                           void *stream);
+
+/*
+ * Greedy choice per row: tokens[b] = the index of the largest logits[b][:]
+ * (the lowest such index; -0 ranks with +0); then, when pos / ctx_len are not
+ * NULL, pos[b] += 1 and ctx_len[b] += 1 (the step's state advance).
+ * logits [B][N] fp32; tokens, pos, ctx_len [B] int32 device arrays.
+ */
+I4_API int i4_argmax_rows(const float *logits, int32_t *tokens, int32_t *pos, int32_t *ctx_len, int B, int N,
+                          void *stream);
 
 /* ---------------------------------------------------------------- decode step */
 

@@ -69,6 +69,10 @@ _SIGS = {
     "paged_gqa_decode_ws_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "paged_gqa_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "paged_gqa_decode_static": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "i4_paged_gqa_decode_strided": (_i, [_vp, ctypes.c_longlong, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                         _f, _vp, _sz, _vp]),
+    "i4_embed_gather": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
+    "i4_argmax_rows": (_i, [_vp, _vp, _vp, _vp, _i, _i, _vp]),
     "i4_paged_gather": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "rmsnorm_rope": (_i, [ctypes.POINTER(RmsnormRopeArgs), _vp]),
     "i4_rmsnorm": (_i, [_vp, _vp, _vp, _vp, _i, _i, _f, _vp]),
@@ -198,6 +202,35 @@ def paged_gqa_decode_static(q, k_pool, v_pool, page_table, ctx_len, out=None, sc
     return out
 
 
+def paged_gqa_decode_strided(q, q_stride: int, Hq: int, k_pool, v_pool, page_table, ctx_len, out, ws, scale=None,
+                             stream=None):
+    """paged_gqa_decode reading the q rows of sequence b at q[b * q_stride ...] (e.g. inside qkv rows)."""
+    B = page_table.shape[0]
+    _, Hkv, P, D = k_pool.shape
+    scale = 1.0 / D ** 0.5 if scale is None else scale
+    _check(lib().i4_paged_gqa_decode_strided(_p(q), int(q_stride), _p(k_pool), _p(v_pool), _p(page_table),
+                                             _p(ctx_len), _p(out), B, Hq, Hkv, D, P, page_table.shape[1],
+                                             float(scale), _p(ws), ws.numel() * ws.element_size(),
+                                             _stream(stream)), "i4_paged_gqa_decode_strided")
+    return out
+
+
+def embed_gather(table, tokens, out, stream=None):
+    """out[b] = table[tokens[b]] (token ids clamped to the table)."""
+    V, H = table.shape
+    _check(lib().i4_embed_gather(_p(table), _p(tokens), _p(out), tokens.numel(), H, V, _stream(stream)),
+           "i4_embed_gather")
+    return out
+
+
+def argmax_rows(logits, tokens, pos=None, ctx_len=None, stream=None):
+    """tokens[b] = argmax(logits[b]) (lowest index on ties); pos and ctx_len advance by one when given."""
+    B, N = logits.shape
+    _check(lib().i4_argmax_rows(_p(logits), _p(tokens), _p(pos), _p(ctx_len), B, N, _stream(stream)),
+           "i4_argmax_rows")
+    return tokens
+
+
 def paged_gather(pool, page_table, ctx_len, max_ctx: int, out=None, stream=None):
     import torch
     _, Hkv, P, D = pool.shape
@@ -244,4 +277,4 @@ def silu_mul(gate_up, out=None, stream=None):
     return out if gate_up.dim() == 2 else out.view(-1)
 
 
-from .runtime import DecodeGraph, DeviceModel, Sequence  # noqa: E402,F401
+from .runtime import BatchedDecode, DecodeGraph, DeviceModel, Sequence  # noqa: E402,F401

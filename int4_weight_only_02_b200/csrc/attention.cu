@@ -285,7 +285,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) paged_gqa_decode_kernel(
     const int gq = lane >> 2, tig = lane & 3;  // MMA group (row) and thread-in-group
     uint32_t qa[8][2];
     {
-        const uint32_t *qrow = reinterpret_cast<const uint32_t *>(p.q + ((size_t)b * p.Hq + g * G + gq) * kHeadDim);
+        const uint32_t *qrow =
+            reinterpret_cast<const uint32_t *>(p.q + (size_t)b * p.q_stride + (size_t)(g * G + gq) * kHeadDim);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             qa[kk][0] = gq < G ? qrow[8 * kk + tig] : 0u;
@@ -592,10 +593,10 @@ extern "C" size_t paged_gqa_decode_ws_bytes(int B, int Hq, int Hkv, int D, int p
     return attn_ws_layout(B, Hq, Hkv, page_size, max_pages_per_seq).bytes;
 }
 
-extern "C" int paged_gqa_decode(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_pool,
-                                const int32_t *page_table, const int32_t *ctx_len, uint16_t *out, int B, int Hq,
-                                int Hkv, int D, int page_size, int max_pages_per_seq, float scale, void *ws,
-                                size_t ws_bytes, void *stream) {
+static int decode_attention(const uint16_t *q, long long q_stride, const uint16_t *k_pool, const uint16_t *v_pool,
+                            const int32_t *page_table, const int32_t *ctx_len, uint16_t *out, int B, int Hq, int Hkv,
+                            int D, int page_size, int max_pages_per_seq, float scale, void *ws, size_t ws_bytes,
+                            void *stream) {
     int st = attn_check(q, k_pool, v_pool, page_table, ctx_len, out, B, Hq, Hkv, D, page_size, max_pages_per_seq);
     if (st) return st;
     const AttnWs L = attn_ws_layout(B, Hq, Hkv, page_size, max_pages_per_seq);
@@ -611,6 +612,7 @@ extern "C" int paged_gqa_decode(const uint16_t *q, const uint16_t *k_pool, const
     p.out = out;
     p.B = B;
     p.Hq = Hq;
+    p.q_stride = q_stride;
     p.Hkv = Hkv;
     p.page_size = page_size;
     p.max_pages = max_pages_per_seq;
@@ -622,6 +624,26 @@ extern "C" int paged_gqa_decode(const uint16_t *q, const uint16_t *k_pool, const
     p.ml_off = L.ml_off;
     p.acc_off = L.acc_off;
     return launch_paged_gqa_decode(p, (cudaStream_t)stream, false);
+}
+
+extern "C" int paged_gqa_decode(const uint16_t *q, const uint16_t *k_pool, const uint16_t *v_pool,
+                                const int32_t *page_table, const int32_t *ctx_len, uint16_t *out, int B, int Hq,
+                                int Hkv, int D, int page_size, int max_pages_per_seq, float scale, void *ws,
+                                size_t ws_bytes, void *stream) {
+    return decode_attention(q, (long long)Hq * D, k_pool, v_pool, page_table, ctx_len, out, B, Hq, Hkv, D, page_size,
+                            max_pages_per_seq, scale, ws, ws_bytes, stream);
+}
+
+extern "C" int i4_paged_gqa_decode_strided(const uint16_t *q, long long q_stride, const uint16_t *k_pool,
+                                           const uint16_t *v_pool, const int32_t *page_table, const int32_t *ctx_len,
+                                           uint16_t *out, int B, int Hq, int Hkv, int D, int page_size,
+                                           int max_pages_per_seq, float scale, void *ws, size_t ws_bytes,
+                                           void *stream) {
+    if (q_stride < (long long)Hq * D || q_stride % 8)
+        return fail(I4_EINVAL, "i4_paged_gqa_decode_strided: q_stride %lld must be >= Hq*D and a multiple of 8",
+                    q_stride);
+    return decode_attention(q, q_stride, k_pool, v_pool, page_table, ctx_len, out, B, Hq, Hkv, D, page_size,
+                            max_pages_per_seq, scale, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------- no-allocation variant
@@ -682,6 +704,7 @@ extern "C" int paged_gqa_decode_static(const uint16_t *q, const uint16_t *k_pool
     p.out = out;
     p.B = B;
     p.Hq = Hq;
+    p.q_stride = (long long)Hq * 128;
     p.Hkv = Hkv;
     p.page_size = page_size;
     p.max_pages = max_pages_per_seq;

@@ -10,6 +10,7 @@ struct AttnParams {
     const int32_t *page_table, *ctx_len;
     uint16_t *out;
     int B, Hq, Hkv, page_size, max_pages;
+    long long q_stride;   // elements between the q rows of consecutive sequences (Hq * 128 when packed)
     int splits, cluster;  // grid x (a multiple of cluster) and CTAs per cluster along x
     float scale;
     char *ws;

@@ -115,6 +115,7 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
             p.out = g->attn;
             p.B = 1;
             p.Hq = d.n_q_heads;
+            p.q_stride = (long long)d.n_q_heads * D;
             p.Hkv = d.n_kv_heads;
             p.page_size = d.page_size;
             p.max_pages = max_pages;

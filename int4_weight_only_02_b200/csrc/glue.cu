@@ -8,6 +8,7 @@
 // same per-element arithmetic as the fused forms.
 #include "common.cuh"
 #include "gemv.cuh"
+#include "gemv_parts.cuh"  // argmax_key
 
 namespace i4 {
 
@@ -114,6 +115,45 @@ __global__ void rope_table_kernel(float2 *cs, int max_ctx, int d, double theta) 
         cs[idx] = rope_cos_sin(idx / half, idx % half, d, theta);
 }
 
+// out[b][:] = table[clamp(tokens[b])][:], one CTA per row, 16-byte copies
+__global__ void embed_gather_kernel(const uint16_t *table, const int32_t *tokens, uint16_t *out, int H, int vocab) {
+    grid_dep_wait();
+    const int b = blockIdx.x;
+    int t = tokens[b];
+    t = t < 0 ? 0 : (t >= vocab ? vocab - 1 : t);
+    const uint4 *src = reinterpret_cast<const uint4 *>(table + (size_t)t * H);
+    uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)b * H);
+    for (int c = threadIdx.x; c < H / 8; c += blockDim.x) dst[c] = src[c];
+}
+
+// tokens[b] = argmax of logits[b][:] (lowest index among equal maxima, -0 ranks with +0); then, when
+// given, pos[b] += 1 and ctx_len[b] += 1. One CTA per row.
+__global__ void __launch_bounds__(256) argmax_rows_kernel(const float *logits, int32_t *tokens, int32_t *pos,
+                                                          int32_t *ctx_len, int N) {
+    grid_dep_wait();
+    __shared__ unsigned long long best[8];
+    const int b = blockIdx.x;
+    const float *row = logits + (size_t)b * N;
+    unsigned long long k = 0ull;
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+        const unsigned long long c = argmax_key(row[i], i);
+        k = c > k ? c : k;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, k, o);
+        k = other > k ? other : k;
+    }
+    if ((threadIdx.x & 31) == 0) best[threadIdx.x >> 5] = k;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) k = best[w] > k ? best[w] : k;
+        tokens[b] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+        if (pos) pos[b] += 1;
+        if (ctx_len) ctx_len[b] += 1;
+    }
+}
+
 int launch_rope_table(float2 *cs, int max_ctx, int d, double theta, cudaStream_t stream) {
     rope_table_kernel<<<256, 256, 0, stream>>>(cs, max_ctx, d, theta);
     return launch_check("rope table");
@@ -167,4 +207,21 @@ extern "C" int silu_mul(const uint16_t *gate_up, uint16_t *out, int M, int I, vo
     const int grid = (int)((n + 255) / 256 < 4 * kNumSMs ? (n + 255) / 256 : 4 * kNumSMs);
     silu_mul_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(gate_up, out, M, I);
     return launch_check("silu_mul");
+}
+
+extern "C" int i4_embed_gather(const uint16_t *table, const int32_t *tokens, uint16_t *out, int B, int H, int vocab,
+                               void *stream) {
+    if (!table || !tokens || !out) return fail(I4_EINVAL, "i4_embed_gather: null pointer");
+    if (B < 1 || B > 65535 || H < 8 || H % 8 || vocab < 1) return fail(I4_EINVAL, "i4_embed_gather: bad sizes");
+    if (!aligned(table, 16) || !aligned(out, 16)) return fail(I4_EALIGN, "i4_embed_gather: 16-byte alignment required");
+    embed_gather_kernel<<<B, 256, 0, (cudaStream_t)stream>>>(table, tokens, out, H, vocab);
+    return launch_check("i4_embed_gather");
+}
+
+extern "C" int i4_argmax_rows(const float *logits, int32_t *tokens, int32_t *pos, int32_t *ctx_len, int B, int N,
+                              void *stream) {
+    if (!logits || !tokens) return fail(I4_EINVAL, "i4_argmax_rows: null pointer");
+    if (B < 1 || B > 65535 || N < 1) return fail(I4_EINVAL, "i4_argmax_rows: bad sizes");
+    argmax_rows_kernel<<<B, 256, 0, (cudaStream_t)stream>>>(logits, tokens, pos, ctx_len, N);
+    return launch_check("i4_argmax_rows");
 }

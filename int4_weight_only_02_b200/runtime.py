@@ -149,3 +149,97 @@ class DecodeGraph:
             self.close()
         except Exception:
             pass
+
+
+class BatchedDecode:
+    """B sequences decoded together: one step is a CUDA graph of library calls -- embedding gather,
+    batched INT4 GEMVs (the B vectors as tensor-core columns where the shape allows), batched
+    RMSNorm (+ residual), RoPE + K/V append, B-sequence paged attention reading q inside the qkv
+    rows, SiLU-mul, lm_head and a per-row argmax that advances each sequence's position.
+    Every sequence has its own page-table row over per-layer pools shared by the batch.
+    """
+
+    def __init__(self, model: DeviceModel, page_tables: np.ndarray, num_pages: int):
+        import torch
+        from . import paged_gqa_decode_ws_bytes
+        s, dev = model.shape, model.device
+        self.model, self.shape = model, s
+        self.B = B = int(page_tables.shape[0])
+        self.page_tables = to_device(np.asarray(page_tables, dtype=np.int32), dev)
+        kv = (int(num_pages), s.n_kv, s.page_size, s.head_dim)
+        self.k_pools = [torch.zeros(kv, dtype=torch.float16, device=dev) for _ in range(s.layers)]
+        self.v_pools = [torch.zeros(kv, dtype=torch.float16, device=dev) for _ in range(s.layers)]
+        i32 = dict(dtype=torch.int32, device=dev)
+        f16 = dict(dtype=torch.float16, device=dev)
+        self.tokens = torch.zeros(B, **i32)
+        self.pos = torch.zeros(B, **i32)
+        self.ctx_len = torch.ones(B, **i32)
+        nqkv = (s.n_q + 2 * s.n_kv) * s.head_dim
+        self.r = torch.zeros((B, s.hidden), **f16)
+        self.xn = torch.zeros((B, s.hidden), **f16)
+        self.qkv = torch.zeros((B, nqkv), **f16)
+        self.attn = torch.zeros((B, s.n_q * s.head_dim), **f16)
+        self.y = torch.zeros((B, s.hidden), **f16)
+        self.gu = torch.zeros((B, 2 * s.inter), **f16)
+        self.mlp = torch.zeros((B, s.inter), **f16)
+        self.logits = torch.zeros((B, s.vocab), dtype=torch.float32, device=dev)
+        nbytes = paged_gqa_decode_ws_bytes(B, s.n_q, s.n_kv, s.head_dim, s.page_size, page_tables.shape[1])
+        self.attn_ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        self.graph = None
+        # vectors per down-projection call: the batched tensor-core GEMV takes rows of up to 4096 weights;
+        # longer rows go through the register kernel, whose x stage holds a power-of-two number of vectors
+        # at 68 bytes per 32 weights each, within 200 KB
+        self.down_rows = B
+        if s.inter > 4096:
+            mr = 1
+            while mr * 2 <= B and mr * 2 * (s.inter // 32) * 68 <= 200 * 1024:
+                mr *= 2
+            self.down_rows = mr
+
+    def reset(self, first_tokens):
+        """Position 0 of every sequence, with the given first tokens."""
+        import torch
+        self.tokens.copy_(torch.as_tensor(np.asarray(first_tokens, dtype=np.int32)))
+        self.pos.zero_()
+        self.ctx_len.fill_(1)
+
+    def step(self, stream=None):
+        """Enqueue one decode step of all B sequences on `stream` (no allocation, capturable)."""
+        from . import (argmax_rows, embed_gather, int4_gemv, paged_gqa_decode_strided, rmsnorm,
+                       rope_kv_append, silu_mul)
+        m, s = self.model, self.shape
+        g, L = m.glob, m.layers
+        nqkv = (s.n_q + 2 * s.n_kv) * s.head_dim
+        embed_gather(g["embed"], self.tokens, self.r, stream=stream)
+        rmsnorm(self.r, L[0]["ln_in"], out=self.xn, eps=s.eps, stream=stream)
+        for li, lw in enumerate(L):
+            int4_gemv(lw["w_qkv"], lw["s_qkv"], self.xn, lw["b_qkv"], y=self.qkv, stream=stream)
+            rope_kv_append(self.qkv, self.pos, s.n_q, s.n_kv, s.theta, self.k_pools[li], self.v_pools[li],
+                           self.page_tables, stream=stream)
+            paged_gqa_decode_strided(self.qkv, nqkv, s.n_q, self.k_pools[li], self.v_pools[li], self.page_tables,
+                                     self.ctx_len, self.attn, self.attn_ws, stream=stream)
+            int4_gemv(lw["w_o"], lw["s_o"], self.attn, y=self.y, stream=stream)
+            rmsnorm(self.y, lw["ln_post"], out=self.xn, resid=self.r, eps=s.eps, stream=stream)
+            int4_gemv(lw["w_gu"], lw["s_gu"], self.xn, y=self.gu, stream=stream)
+            silu_mul(self.gu, out=self.mlp, stream=stream)
+            for m0 in range(0, self.B, self.down_rows):  # rows beyond 4096 weights: the x stage holds <= 4 vectors
+                int4_gemv(lw["w_d"], lw["s_d"], self.mlp[m0:m0 + self.down_rows], y=self.y[m0:m0 + self.down_rows],
+                          stream=stream)
+            gamma = L[li + 1]["ln_in"] if li + 1 < len(L) else g["ln_final"]
+            rmsnorm(self.y, gamma, out=self.xn, resid=self.r, eps=s.eps, stream=stream)
+        int4_gemv(g["w_lm"], g["s_lm"], self.xn, y=self.logits, out_fp32=True, stream=stream)
+        argmax_rows(self.logits, self.tokens, self.pos, self.ctx_len, stream=stream)
+
+    def capture(self):
+        """Capture one step as a CUDA graph (after one eager step has configured every kernel)."""
+        import torch
+        side = torch.cuda.Stream()
+        self.graph = torch.cuda.CUDAGraph()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(self.graph, stream=side):
+                self.step(stream=side)
+        torch.cuda.synchronize()
+
+    def replay(self):
+        self.graph.replay()
