@@ -67,7 +67,7 @@ I4_API const char *i4_version(void);
  *   y      [M][N], 4-byte aligned for fp32.
  * Requires group == 128, K % 128 == 0, K <= 32768, 1 <= M <= 8, N >= 1; shapes
  * off the tensor-core paths stage the M vectors in shared memory, which allows
- * M <= 8 up to K = 11904 and M <= 4 up to K = 24064 (larger M * K is refused
+ * M <= 8 up to K = 12032 and M <= 4 up to K = 24064 (larger M * K is refused
  * with I4_EUNSUPPORTED). The kernel is chosen by the "unpack" option below.
  */
 I4_API int int4_gemv(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
