@@ -59,6 +59,25 @@ def test_host_validation_without_gpu(i4lib):
     assert L.i4_set_option(b"nonsense", 1) == i4lib.I4_EINVAL
 
 
+def test_batched_decode_entries_validate_without_gpu(i4lib):
+    L = i4lib.lib()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    # q rows closer than Hq * D, or not a multiple of 8 elements apart
+    assert L.i4_paged_gqa_decode_strided(fake, 28 * 128 - 8, fake, fake, fake, fake, fake, 2, 28, 4, 128, 16, 4,
+                                         1.0, fake, 1 << 20, None) == i4lib.I4_EINVAL
+    assert L.i4_paged_gqa_decode_strided(fake, 4608 + 4, fake, fake, fake, fake, fake, 2, 28, 4, 128, 16, 4,
+                                         1.0, fake, 1 << 20, None) == i4lib.I4_EINVAL
+    assert b"q_stride" in L.i4_last_error()
+    # the strided entry applies paged_gqa_decode's checks too
+    assert L.i4_paged_gqa_decode_strided(fake, 4608, fake, fake, fake, fake, fake, 2, 28, 4, 128, 12, 4,
+                                         1.0, fake, 1 << 20, None) == i4lib.I4_EUNSUPPORTED
+    assert L.i4_embed_gather(None, fake, fake, 2, 64, 10, None) == i4lib.I4_EINVAL
+    assert L.i4_embed_gather(fake, fake, fake, 2, 60, 10, None) == i4lib.I4_EINVAL       # H % 8
+    assert L.i4_embed_gather(ctypes.c_void_p((1 << 20) + 2), fake, fake, 2, 64, 10, None) == i4lib.I4_EALIGN
+    assert L.i4_argmax_rows(fake, fake, None, None, 0, 10, None) == i4lib.I4_EINVAL
+    assert L.i4_argmax_rows(None, fake, None, None, 1, 10, None) == i4lib.I4_EINVAL
+
+
 def test_graph_create_validation_without_gpu(i4lib):
     desc = i4lib.ModelDesc(28, 3584, 18944, 28, 4, 64, 152064, 128, 16, 4096, 1e6, 1e-6)
     handle = ctypes.c_void_p()
