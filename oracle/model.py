@@ -17,6 +17,12 @@ A prompt may be fed a whole block of tokens at once: every row of the block
 goes through exactly the elementwise operations of a one-token step, and
 token i only reads K/V up to its own position, so the result is the same as
 feeding the tokens one by one (``tests/test_oracle_model.py`` checks this).
+
+Pins: the parts are pinned in ``tests/test_oracle_primitives.py``; the
+composition is pinned by the block-prompt identity, the K/V page placement and
+two closed-form special cases (zero o/down projections; zero queries) in
+``tests/test_oracle_model.py``. The general composition with every branch active
+has no independent reference: parity unpinned beyond those cases.
 """
 from __future__ import annotations
 
