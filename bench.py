@@ -20,6 +20,13 @@ timed region, and the CPU oracle timed on a bounded sample.
 
 --impl reference times the CPU oracle instead (rank 0 only), each step one
 decoder layer of one token at context 513, scaled to tok/s.
+
+Other modes (one JSON line per case, not the benchmark line):
+  --profile-kernel NAME  one kernel of a one-layer model, for ncu captures;
+  --attention-sweep      paged attention over contexts 512-32768, page sizes 16/64,
+                         batches 1/8/32 with ragged lengths (KV GB/s, L2-cold);
+  --gemv-batch           the gate/up GEMV for 1, 2, 4 and 8 vectors (weight GB/s);
+  --batched-decode B     B sequences decoded together (tok/s over the batch).
 """
 from __future__ import annotations
 
