@@ -445,6 +445,50 @@ def run_batched_decode(args):
     return 0
 
 
+def run_prefill(args):
+    """Time to first token of the 7B-shape decoder for a 512-token prompt, prefilled 8 positions per
+    step through the batched library calls (causal over one sequence's pages), against the same prompt
+    fed one token per step through the fused decode graph. One JSON line."""
+    import numpy as np
+    import torch
+
+    import int4_weight_only_02_b200 as i4
+    from int4_weight_only_02_b200 import synth
+    dev = torch.device("cuda", 0)
+    shape = synth.QWEN7B
+    B = args.prefill
+    model = i4.DeviceModel.synthetic(shape, device=dev)
+    table = synth.page_table(shape, 0)
+    prompt = synth.prompt_tokens(shape, args.prompt, seed=0)
+    bd = i4.BatchedDecode(model, np.tile(table, (B, 1)), num_pages=shape.max_pages)
+    bd.prefill(prompt)  # warm-up (captures the step graph)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    tok = bd.prefill(prompt)
+    e1.record()
+    torch.cuda.synchronize()
+    chunked_ms = e0.elapsed_time(e1)
+    seq = i4.Sequence(model, table, prompt)
+    graph = i4.DecodeGraph(model, seq)
+    for _ in range(len(prompt)):
+        graph.replay()
+    torch.cuda.synchronize()
+    seq.reset()
+    e0.record()
+    for _ in range(len(prompt)):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    token_ms = e0.elapsed_time(e1)
+    first = int(seq.history[len(prompt)].item())
+    graph.close()
+    print(json.dumps({"prefill": B, "prompt": len(prompt), "ttft_ms_chunked": round(chunked_ms, 2),
+                      "ttft_ms_token_by_token": round(token_ms, 2), "first_token_chunked": tok,
+                      "first_token_graph": first, "device_error": i4.device_error()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -466,6 +510,8 @@ def main():
     ap.add_argument("--attention-sweep", action="store_true",
                     help="paged attention sweep over contexts, page sizes 16/64 and batches 1/8/32 (KV GB/s)")
     ap.add_argument("--sweep-contexts", default="512,2048,8192,32768")
+    ap.add_argument("--prefill", type=int, default=0,
+                    help="time to first token with this many prompt positions per step (e.g. 8)")
     ap.add_argument("--batched-decode", type=int, default=0,
                     help="decode this many sequences together (1..8) through the batched library calls")
     ap.add_argument("--gemv-batch", action="store_true",
@@ -481,6 +527,8 @@ def main():
         return run_gemv_batch(args)
     if args.batched_decode:
         return run_batched_decode(args)
+    if args.prefill:
+        return run_prefill(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
 

@@ -243,3 +243,34 @@ class BatchedDecode:
 
     def replay(self):
         self.graph.replay()
+
+    def prefill(self, prompt, graph: bool = True) -> int:
+        """Causal prefill of ONE sequence, B prompt tokens per step: every row of the batch is one prompt
+        position of the same sequence (all page-table rows must be equal), row b at position c + b with
+        context c + b + 1, so attention over the shared pages is causal and the K/V of the whole chunk land
+        before any row reads them. len(prompt) must be a multiple of B. Returns the first generated token
+        (the argmax at the last prompt position)."""
+        import torch
+        prompt = np.asarray(prompt, dtype=np.int32)
+        B, n = self.B, len(prompt)
+        if n % B:
+            raise ValueError(f"prompt length {n} is not a multiple of the batch {B}")
+        if graph and self.graph is None:
+            self._prefill_chunk(prompt[:B], 0)
+            self.step()
+            torch.cuda.synchronize()
+            self.capture()
+            start = B
+        else:
+            start = 0
+        for c in range(start, n, B):
+            self._prefill_chunk(prompt[c:c + B], c)
+            self.replay() if graph else self.step()
+        torch.cuda.synchronize()
+        return int(self.tokens[B - 1].item())
+
+    def _prefill_chunk(self, tokens, c: int):
+        import torch
+        self.tokens.copy_(torch.from_numpy(np.ascontiguousarray(tokens)))
+        self.pos.copy_(torch.arange(c, c + self.B, dtype=torch.int32))
+        self.ctx_len.copy_(torch.arange(c + 1, c + self.B + 1, dtype=torch.int32))

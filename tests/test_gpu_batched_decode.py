@@ -71,3 +71,26 @@ def test_embed_gather_and_argmax_rows(i4lib, cuda):
     want = [oracle.argmax(logits[b]) for b in range(4)]
     assert tok.cpu().tolist() == want
     assert pos.cpu().tolist() == [1, 2, 3, 4] and ctx.cpu().tolist() == [2, 3, 4, 5]
+
+
+def test_chunked_prefill_matches_oracle(i4lib, cuda):
+    """Prefill of one sequence 8 positions per step (rows = consecutive positions over one page-table
+    row): the first generated token and the last position's logits equal the oracle's."""
+    import torch
+    shape = synth.ModelShape(layers=2, hidden=512, inter=1024, n_q=4, n_kv=2, head_dim=128, vocab=1000, group=128,
+                             page_size=16, max_ctx=64)
+    layers = [synth.layer_weights(shape, i, 1) for i in range(shape.layers)]
+    glob = synth.global_weights(shape, 1)
+    prompt = synth.prompt_tokens(shape, 24, seed=5)
+    table = synth.page_table(shape, 2)
+    dec = oracle.DecoderOracle(shape, layers, glob, table)
+    want_logits, _ = dec.forward(prompt, 0)
+    want = oracle.argmax(want_logits)
+
+    model = i4lib.DeviceModel(shape, layers, glob, device=cuda)
+    bd = i4lib.BatchedDecode(model, np.tile(table, (8, 1)), num_pages=shape.max_pages)
+    got = bd.prefill(prompt)
+    assert got == want
+    got_logits = bd.logits[7].cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(got_logits - want_logits)) / np.max(np.abs(want_logits)) <= 1e-2
+    assert i4lib.device_error() == 0
