@@ -26,7 +26,8 @@ Other modes (one JSON line per case, not the benchmark line):
   --attention-sweep      paged attention over contexts 512-32768, page sizes 16/64,
                          batches 1/8/32 with ragged lengths (KV GB/s, L2-cold);
   --gemv-batch           the gate/up GEMV for 1, 2, 4 and 8 vectors (weight GB/s);
-  --batched-decode B     B sequences decoded together (tok/s over the batch).
+  --batched-decode B     B sequences decoded together (tok/s over the batch);
+  --prefill B            time to first token with B prompt positions per step.
 """
 from __future__ import annotations
 
