@@ -45,8 +45,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode tok/s at batch 1 (7B-shape INT4); INT4 GEMV HBM GB/s vs B200 peak"
 WORKLOAD = ("qwen2.5-7b-shape decoder (28 layers, hidden 3584, mlp 18944, 28q/4kv heads, head_dim 128, "
-            "vocab 152064), int4 group-128 fp16-scale weights, batch 1, 512-token prompt then greedy decode, "
-            "paged KV page 16, one CUDA graph per token")
+            "vocab 152064), int4 group-128 fp16-scale weights (codes uniform in [-8, 7], |scale| uniform in "
+            "[0.005, 0.02] with a random sign per group: all-positive scales overflow the fp16 residual in "
+            "layer 1), batch 1, 512-token prompt then greedy decode, paged KV page 16, one CUDA graph per token")
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
@@ -141,72 +142,123 @@ def traffic_from_profile(profile: str, names):
         return None
 
 
-def oracle_cpu_sample(shape, layers_np, glob_np, n_tokens: int = 8):
-    """The CPU oracle as it stands: n_tokens decode steps at position 512 with the KV
-    cache below it filled with random fp16 values."""
+def primed_oracle(shape, layers_np, glob_np, first_pos: int, n_tokens: int):
+    """The CPU oracle decoder with the KV cache below `first_pos` filled with seeded random fp16 values
+    (N(0, 4^2), the spread of the model's own K/V), ready to decode tokens at first_pos, first_pos + 1, ..."""
     import numpy as np
 
     import oracle
     from int4_weight_only_02_b200 import synth
     dec = oracle.DecoderOracle(shape, layers_np, glob_np, synth.page_table(shape, 0), num_pages=shape.max_pages)
     rng = np.random.default_rng(123)
-    used = (512 + n_tokens + shape.page_size - 1) // shape.page_size
+    used = (first_pos + n_tokens + shape.page_size - 1) // shape.page_size
     for li in range(shape.layers):
         for pool in (dec.k_pools[li], dec.v_pools[li]):
             for p in dec.page_table[:used]:
                 pool[p] = (rng.standard_normal(pool[p].shape) * 4).astype(np.float16)
+    return dec
+
+
+def oracle_cpu_sample(shape, layers_np, glob_np, n_tokens: int = 8):
+    """The CPU oracle as it stands: n_tokens full decode steps at positions 512.. (bounded sample)."""
+    import oracle
+    dec = primed_oracle(shape, layers_np, glob_np, 512, n_tokens)
+    threads = oracle.set_threads(0)
     t0 = time.perf_counter()
     tok = 1
     for i in range(n_tokens):
         logits, _ = dec.forward([tok], 512 + i)
         tok = oracle.argmax(logits)
     el = time.perf_counter() - t0
-    return {"value": round(n_tokens / el, 4), "unit": "tok/s", "cores": os.cpu_count(), "kind": "oracle",
+    return {"value": round(n_tokens / el, 4), "unit": "tok/s", "cores": threads, "host_cpus": os.cpu_count(),
+            "kind": "oracle",
             "sample": f"{n_tokens} full decode tokens (28 layers + lm_head) at positions 512..{511 + n_tokens}, "
-                      f"KV below filled with random fp16, fp64 C/numpy oracle on all host cores "
+                      f"KV below filled with random fp16, fp64 C/numpy oracle, {threads} OpenMP threads "
                       f"({el:.1f} s)"}
 
 
-def run_reference(args):
-    """CPU oracle arm: each step is one decoder layer of one token at context 513."""
-    if int(os.environ.get("RANK", "0")) != 0:
-        return 0
+def oracle_unit_configs():
+    """The unit workloads timed on the CPU oracle, one thread (pinned to one core) and all threads:
+    qkv INT4 GEMV (K 3584, N 4608), paged attention (28/4 heads, ctx 512, page 16), MLP block
+    (RMSNorm, gate/up GEMV, SiLU-mul, down GEMV); ms and algorithmic GB/s of each."""
     import numpy as np
 
     import oracle
     from int4_weight_only_02_b200 import synth
+    w, s, x, b = synth.gemv_case(4608, 3584, seed=0, bias=True)
+    q, kp, vp, table, ctx = synth.attention_case([512], page_size=16, seed=0)
+    mw_gu, ms_gu, mx, _ = synth.gemv_case(37888, 3584, seed=0)
+    mw_d, ms_d, _, _ = synth.gemv_case(3584, 18944, seed=0)
+    gamma = synth.normal_f16(synth.rng_for(0, 77), (3584,), 1.0, 0.1)
+    units = {
+        "C0a_qkv_gemv": (lambda: oracle.int4_gemv(w, s, x[0], b), 4608 * 1792 + 4608 * 28 * 2),
+        "C0b_attention_ctx512": (lambda: oracle.paged_attention(q[0], kp, vp, table[0], 512), 512 * 4 * 128 * 2 * 2),
+        "C1_mlp_block": (lambda: oracle.int4_gemv(mw_d, ms_d, oracle.silu_mul(
+            *np.split(oracle.int4_gemv(mw_gu, ms_gu, oracle.rmsnorm(mx[0], gamma, 1e-6)), 2))),
+            37888 * 1792 + 37888 * 28 * 2 + 3584 * 9472 + 3584 * 148 * 2),
+    }
+    all_threads = oracle.set_threads(0)
+    out = {"nproc": os.cpu_count(), "threads_all": all_threads}
+    try:
+        aff = os.sched_getaffinity(0)
+    except AttributeError:
+        aff = None
+    for name, (fn, nbytes) in units.items():
+        rec = {"bytes": nbytes}
+        for label, threads in (("one_thread", 1), ("all_threads", all_threads)):
+            oracle.set_threads(threads)
+            if threads == 1 and aff:
+                os.sched_setaffinity(0, {min(aff)})
+            try:
+                fn()
+                reps, t0 = 0, time.perf_counter()
+                while reps < 3 or time.perf_counter() - t0 < 0.5:
+                    fn()
+                    reps += 1
+                ms = (time.perf_counter() - t0) / reps * 1e3
+            finally:
+                if aff:
+                    os.sched_setaffinity(0, aff)
+            rec[label] = {"ms": round(ms, 3), "GBs": round(nbytes / (ms * 1e-3) / 1e9, 3)}
+        out[name] = rec
+    oracle.set_threads(all_threads)
+    return out
+
+
+def run_reference(args):
+    """CPU oracle arm: each step is one full decode token of the same workload (28 layers, final norm,
+    lm_head, argmax) at positions 512, 513, ... after a KV cache of seeded random values; tok/s =
+    steps / the timed steps' total time."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    import oracle
+    from int4_weight_only_02_b200 import synth
     shape = synth.QWEN7B
-    one = synth.ModelShape(layers=1)
-    lw = [synth.layer_weights(shape, 0, 0)]
+    layers = [synth.layer_weights(shape, i, 0) for i in range(shape.layers)]
     glob = synth.global_weights(shape, 0)
-    dec = oracle.DecoderOracle(one, lw, glob, synth.page_table(shape, 0), num_pages=shape.max_pages)
-    rng = np.random.default_rng(5)
-    for pool in (dec.k_pools[0], dec.v_pools[0]):
-        for p in dec.page_table[:33]:
-            pool[p] = (rng.standard_normal(pool[p].shape) * 4).astype(np.float16)
-    r = glob["embed"][[7]].astype(np.float16)
-    t0 = time.perf_counter()
-    x = oracle.rmsnorm(r[-1], glob["ln_final"], shape.eps)
-    oracle.int4_gemv(glob["w_lm"], glob["s_lm"], x, None, shape.group, np.float32)
-    t_lm = time.perf_counter() - t0
+    dec = primed_oracle(shape, layers, glob, 512, args.warmup + args.steps)
+    threads = oracle.set_threads(0)
+    tok, pos = int(synth.prompt_tokens(shape, 512, 0)[-1]), 512
     for _ in range(args.warmup):
-        dec.layer(0, r, [512])
-    times = []
+        logits, _ = dec.forward([tok], pos)
+        tok, pos = oracle.argmax(logits), pos + 1
+    t0 = time.perf_counter()
     for _ in range(args.steps):
-        t0 = time.perf_counter()
-        dec.layer(0, r, [512])
-        times.append(time.perf_counter() - t0)
-    t_layer = statistics.mean(times)
-    ms_tok = (shape.layers * t_layer + t_lm) * 1e3
-    value = 1e3 / ms_tok
-    sample = (f"each step = one decoder layer of one token at context 513 (fp64 oracle, {os.cpu_count()} host "
-              f"cores); tok/s = 1 / (28 x mean layer time + lm_head time {t_lm * 1e3:.0f} ms)")
+        logits, _ = dec.forward([tok], pos)
+        tok, pos = oracle.argmax(logits), pos + 1
+    el = time.perf_counter() - t0
+    ms_tok = el / args.steps * 1e3
+    value = args.steps / el
+    sample = (f"{args.steps} timed full decode tokens (28 layers + lm_head + argmax) at positions "
+              f"{512 + args.warmup}..{pos - 1} after {args.warmup} warm-up tokens; KV cache below position 512 "
+              f"seeded random fp16; fp64 C/numpy oracle, {threads} OpenMP threads on {os.cpu_count()} host cpus "
+              f"({el:.1f} s timed)")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "tok/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_tok, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "prompt": 512},
-            "cpu_baseline": {"value": round(value, 5), "unit": "tok/s", "cores": os.cpu_count(), "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": round(value, 5), "unit": "tok/s", "cores": threads,
+                             "host_cpus": os.cpu_count(), "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 5), "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -225,6 +277,39 @@ def max_over_ranks(value_ms: float, world: int, device) -> float:
 def job_tokens_per_s(steps: int, world: int, ms_max: float) -> float:
     """Replicas: every rank decodes `steps` tokens of its own sequence; the job rate uses the slowest rank."""
     return world * steps / (ms_max / 1e3)
+
+
+def teacher_forced(i4, model, shape, gold, torch):
+    """The oracle's 128 greedy tokens forced as the input stream after the 512-token prompt: at every step
+    the GPU's argmax against the oracle's token, with the oracle's top-2 gap where they differ, and the
+    first generated step's logits against the oracle's sampled logits."""
+    import numpy as np
+
+    from int4_weight_only_02_b200 import synth
+    prompt = synth.prompt_tokens(shape, gold["n_prompt"], gold["seed"])
+    want = np.asarray(gold["tokens"])
+    gaps = np.asarray(gold["top2_gap"])
+    forced = np.concatenate([prompt, want[:-1]]).astype(np.int32)
+    seq = i4.Sequence(model, synth.page_table(shape, gold["seed"]), forced)
+    g = i4.DecodeGraph(model, seq)
+    for _ in range(len(prompt) - 1):
+        g.replay()
+    picks, first_err = [], None
+    idx = np.asarray(gold["first_logits_sample"]["index"])
+    ref = np.asarray(gold["first_logits_sample"]["value"])
+    for i in range(len(want)):
+        g.replay()
+        lg = seq.logits.cpu().numpy()
+        if i == 0:
+            first_err = float(np.max(np.abs(lg[idx].astype(np.float64) - ref)))
+        picks.append(int(np.flatnonzero(lg == lg.max())[0]))
+    g.close()
+    picks = np.asarray(picks)
+    diff = np.flatnonzero(picks != want)
+    return {"teacher_forced_agree": int(len(want) - diff.size), "teacher_forced_steps": int(len(want)),
+            "teacher_forced_disagree_at": [[int(i), round(float(gaps[i]), 4)] for i in diff],
+            "first_step_max_abs_logit_err": round(first_err, 5),
+            "oracle_gaps_below_0.1": int(np.sum(gaps < 0.1))}
 
 
 PROFILE_KERNELS = {"qkv": 0, "attention": 1, "o": 2, "gate_up": 3, "down": 4, "lm_head": 5}
@@ -484,9 +569,13 @@ def run_prefill(args):
     token_ms = e0.elapsed_time(e1)
     first = int(seq.history[len(prompt)].item())
     graph.close()
+    err = i4.device_error()
     print(json.dumps({"prefill": B, "prompt": len(prompt), "ttft_ms_chunked": round(chunked_ms, 2),
                       "ttft_ms_token_by_token": round(token_ms, 2), "first_token_chunked": tok,
-                      "first_token_graph": first, "device_error": i4.device_error()}), flush=True)
+                      "first_token_graph": first, "device_error": err}), flush=True)
+    if tok != first or err:
+        print(f"prefill: first tokens differ ({tok} vs {first}) or device error {err}", file=sys.stderr)
+        return 1
     return 0
 
 
@@ -623,6 +712,17 @@ def main():
     torch.cuda.synchronize()
     e2e_tok_s = job_tokens_per_s(args.steps, world, max_over_ranks(e0.elapsed_time(e1), world, dev))
 
+    # spread over a longer decode: 8 more chunks of 16 tokens, ms/token of each chunk
+    chunk_ms = []
+    for _ in range(8):
+        e0.record(stream)
+        for _ in range(16):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        chunk_ms.append(e0.elapsed_time(e1) / 16)
+    ctx_spread = int(seq.ctx_len.item()) - 1
+
     # eager launches of the same kernels (the pages' eager-vs-graph comparison)
     torch.cuda.synchronize()
     e0.record(stream)
@@ -707,6 +807,10 @@ def main():
                           "frac_of_8TBs": round(step_gbs / NOMINAL_HBM_GBS, 4),
                           "frac_of_measured": round(step_gbs / peak, 4)},
         "eager_ms_per_step": round(eager_ms, 3),
+        "token_spread": {"tokens": 128, "chunks": 8, "ctx_last": ctx_spread,
+                         "ms_per_token_min": round(min(chunk_ms), 4),
+                         "ms_per_token_median": round(statistics.median(chunk_ms), 4),
+                         "ms_per_token_max": round(max(chunk_ms), 4)},
         "e2e": {"value": round(e2e_tok_s, 2), "unit": "tok/s", "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4},
         "gpu_launches": args.steps * n_k,
         "clocks": clocks.summary(),
@@ -721,6 +825,7 @@ def main():
             same += 1
         line["greedy_vs_oracle"] = {"compared": n, "identical_prefix": same,
                                     "note": "free-running; first difference expected at an oracle top-2 near-tie"}
+        line["greedy_vs_oracle"].update(teacher_forced(i4, model, shape, gold, torch))
     graph.close()
     if world > 1:
         dist.barrier()
@@ -729,6 +834,8 @@ def main():
         if want_cpu:
             del model, seq
             line["cpu_baseline"] = oracle_cpu_sample(shape, layers_np, glob_np)
+            del layers_np, glob_np
+            line["cpu_baseline_units"] = oracle_unit_configs()
         print(json.dumps(line), flush=True)
     return 0
 

@@ -139,6 +139,29 @@ class DecodeGraph:
         """Launch only kernel `index` of the step (benchmarking; see decode_step_launch_kernel)."""
         _check(lib().decode_step_launch_kernel(self._h, index, _stream(stream)), "decode_step_launch_kernel")
 
+    BUFFERS = {"resid": 0, "q": 1, "attn": 2, "mlp": 3}
+
+    def _buffer_len(self, name: str) -> int:
+        s = self.model.shape
+        return {"resid": s.hidden, "q": s.n_q * s.head_dim, "attn": s.n_q * s.head_dim, "mlp": s.inter}[name]
+
+    def read_buffer(self, name: str, stream=None):
+        """Copy of one of the step's activation buffers ('resid', 'q', 'attn', 'mlp') as an fp16 tensor."""
+        import torch
+        out = torch.empty(self._buffer_len(name), dtype=torch.float16, device=self.model.device)
+        _check(lib().decode_step_buffer_copy(self._h, self.BUFFERS[name], _p(out), out.numel() * 2, 0,
+                                             _stream(stream)), "decode_step_buffer_copy")
+        return out
+
+    def write_buffer(self, name: str, values, stream=None):
+        """Overwrite one of the step's activation buffers with fp16 `values` (a device tensor)."""
+        import torch
+        v = values.to(device=self.model.device, dtype=torch.float16).contiguous()
+        assert v.numel() == self._buffer_len(name)
+        _check(lib().decode_step_buffer_copy(self._h, self.BUFFERS[name], _p(v), v.numel() * 2, 1,
+                                             _stream(stream)), "decode_step_buffer_copy")
+        torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+
     def close(self):
         if getattr(self, "_h", None):
             _check(lib().decode_step_graph_destroy(self._h), "decode_step_graph_destroy")
@@ -165,7 +188,8 @@ class BatchedDecode:
         s, dev = model.shape, model.device
         self.model, self.shape = model, s
         self.B = B = int(page_tables.shape[0])
-        self.page_tables = to_device(np.asarray(page_tables, dtype=np.int32), dev)
+        self._tables_np = np.asarray(page_tables, dtype=np.int32).copy()
+        self.page_tables = to_device(self._tables_np, dev)
         kv = (int(num_pages), s.n_kv, s.page_size, s.head_dim)
         self.k_pools = [torch.zeros(kv, dtype=torch.float16, device=dev) for _ in range(s.layers)]
         self.v_pools = [torch.zeros(kv, dtype=torch.float16, device=dev) for _ in range(s.layers)]
@@ -248,13 +272,22 @@ class BatchedDecode:
         """Causal prefill of ONE sequence, B prompt tokens per step: every row of the batch is one prompt
         position of the same sequence (all page-table rows must be equal), row b at position c + b with
         context c + b + 1, so attention over the shared pages is causal and the K/V of the whole chunk land
-        before any row reads them. len(prompt) must be a multiple of B. Returns the first generated token
-        (the argmax at the last prompt position)."""
+        before any row reads them. len(prompt) must be a multiple of B and fit the page-table row. Returns
+        the first generated token (the argmax at the last prompt position).
+
+        Afterwards the K/V of positions 0..n-1 sit in this object's pools and row b of the batch is at
+        position n - B + b + 1; decoding of the sequence continues from position n with
+        ``continue_state(n, first_token)`` (every row then computes the same next token)."""
         import torch
         prompt = np.asarray(prompt, dtype=np.int32)
         B, n = self.B, len(prompt)
         if n % B:
             raise ValueError(f"prompt length {n} is not a multiple of the batch {B}")
+        if not np.all(self._tables_np == self._tables_np[:1]):
+            raise ValueError("prefill needs every page-table row to be the same sequence's row")
+        cap = self._tables_np.shape[1] * self.shape.page_size
+        if n > cap:
+            raise ValueError(f"prompt length {n} exceeds the page-table row ({cap} positions)")
         if graph and self.graph is None:
             self._prefill_chunk(prompt[:B], 0)
             self.step()
@@ -268,6 +301,14 @@ class BatchedDecode:
             self.replay() if graph else self.step()
         torch.cuda.synchronize()
         return int(self.tokens[B - 1].item())
+
+    def continue_state(self, n: int, first_token: int):
+        """After ``prefill`` of n tokens: every row set to decode the same sequence at position n (token
+        first_token, context n + 1) over the K/V the prefill left in this object's pools."""
+        import torch
+        self.tokens.fill_(int(first_token))
+        self.pos.fill_(int(n))
+        self.ctx_len.fill_(int(n) + 1)
 
     def _prefill_chunk(self, tokens, c: int):
         import torch

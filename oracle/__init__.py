@@ -64,6 +64,12 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
+def set_threads(n: int = 0) -> int:
+    """OpenMP threads of the C loops (0 = leave as is); returns the count in effect (results do not depend
+    on it)."""
+    return int(lib().o_set_threads(int(n)))
+
+
 def _p(a: np.ndarray):
     return ctypes.c_void_p(a.ctypes.data) if a is not None else ctypes.c_void_p(0)
 

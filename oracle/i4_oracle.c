@@ -25,6 +25,7 @@
  * in increasing k (or t) order, so results do not depend on the thread count.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -49,6 +50,13 @@ void o_f16_to_f64(const uint16_t *in, int64_t n, double *out) {
 
 void o_f64_to_f16(const double *in, int64_t n, uint16_t *out) {
     for (int64_t i = 0; i < n; ++i) out[i] = double_to_half_bits(in[i]);
+}
+
+/* OpenMP threads of the row and head loops (n > 0 sets it); returns the count in effect. Results do not
+ * depend on it: each output element is still summed by one thread in a fixed order. */
+int o_set_threads(int n) {
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
 }
 
 /* Field i (0..7) of a packed word as a signed integer in [-8, 7]. */

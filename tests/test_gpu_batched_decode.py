@@ -73,15 +73,18 @@ def test_embed_gather_and_argmax_rows(i4lib, cuda):
     assert pos.cpu().tolist() == [1, 2, 3, 4] and ctx.cpu().tolist() == [2, 3, 4, 5]
 
 
-def test_chunked_prefill_matches_oracle(i4lib, cuda):
+@pytest.mark.parametrize("inter,n_prompt,graph", [(1024, 24, True), (1024, 40, False), (4608, 40, True)])
+def test_chunked_prefill_matches_oracle(i4lib, cuda, inter, n_prompt, graph):
     """Prefill of one sequence 8 positions per step (rows = consecutive positions over one page-table
-    row): the first generated token and the last position's logits equal the oracle's."""
+    row): the first generated token and the last position's logits equal the oracle's. Prompts of 3
+    and 5 chunks cross partially filled pages; eager and graph steps; intermediate 4608 sends the
+    down projection through the split 4-vector calls."""
     import torch
-    shape = synth.ModelShape(layers=2, hidden=512, inter=1024, n_q=4, n_kv=2, head_dim=128, vocab=1000, group=128,
-                             page_size=16, max_ctx=64)
+    shape = synth.ModelShape(layers=2, hidden=512, inter=inter, n_q=4, n_kv=2, head_dim=128, vocab=1000,
+                             group=128, page_size=16, max_ctx=64)
     layers = [synth.layer_weights(shape, i, 1) for i in range(shape.layers)]
     glob = synth.global_weights(shape, 1)
-    prompt = synth.prompt_tokens(shape, 24, seed=5)
+    prompt = synth.prompt_tokens(shape, n_prompt, seed=5)
     table = synth.page_table(shape, 2)
     dec = oracle.DecoderOracle(shape, layers, glob, table)
     want_logits, _ = dec.forward(prompt, 0)
@@ -89,8 +92,29 @@ def test_chunked_prefill_matches_oracle(i4lib, cuda):
 
     model = i4lib.DeviceModel(shape, layers, glob, device=cuda)
     bd = i4lib.BatchedDecode(model, np.tile(table, (8, 1)), num_pages=shape.max_pages)
-    got = bd.prefill(prompt)
+    if inter > 4096:
+        assert bd.down_rows < bd.B
+    got = bd.prefill(prompt, graph=graph)
     assert got == want
     got_logits = bd.logits[7].cpu().numpy().astype(np.float64)
     assert np.max(np.abs(got_logits - want_logits)) / np.max(np.abs(want_logits)) <= 1e-2
     assert i4lib.device_error() == 0
+
+
+def test_chunked_prefill_rejects_bad_prompts(i4lib, cuda):
+    shape = synth.ModelShape(layers=1, hidden=512, inter=1024, n_q=4, n_kv=2, head_dim=128, vocab=1000,
+                             group=128, page_size=16, max_ctx=64)
+    layers = [synth.layer_weights(shape, 0, 1)]
+    glob = synth.global_weights(shape, 1)
+    model = i4lib.DeviceModel(shape, layers, glob, device=cuda)
+    table = synth.page_table(shape, 2)
+    bd = i4lib.BatchedDecode(model, np.tile(table, (8, 1)), num_pages=shape.max_pages)
+    with pytest.raises(ValueError, match="multiple"):
+        bd.prefill(np.arange(12, dtype=np.int32))
+    with pytest.raises(ValueError, match="exceeds"):
+        bd.prefill(np.arange(72, dtype=np.int32))
+    other = np.tile(table, (8, 1))
+    other[3] = np.roll(other[3], 1)
+    bd2 = i4lib.BatchedDecode(model, other, num_pages=shape.max_pages)
+    with pytest.raises(ValueError, match="same sequence"):
+        bd2.prefill(np.arange(16, dtype=np.int32))
