@@ -111,7 +111,8 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-GEMV_SOURCES = ["gemv_stream.cu", "gemv_parts.cuh", "gemv.cuh", "common.cuh", "async.cuh"]
+GEMV_SOURCES = ["gemv_stream.cu", "gemv_parts.cuh", "gemv.cuh", "common.cuh", "async.cuh", "mma.cuh"]
+PERSIST_SOURCES = ["persist.cu", "persist.cuh", "gemv_parts.cuh", "gemv.cuh", "common.cuh", "async.cuh", "mma.cuh"]
 
 
 def sources_hash(names) -> str:
@@ -312,7 +313,7 @@ def teacher_forced(i4, model, shape, gold, torch):
             "oracle_gaps_below_0.1": int(np.sum(gaps < 0.1))}
 
 
-PROFILE_KERNELS = {"qkv": 0, "attention": 1, "o": 2, "gate_up": 3, "down": 4, "lm_head": 5}
+PROFILE_KERNELS = {"qkv": 0, "attention": 1, "o": 2, "gate_up": 3, "down": 4, "lm_head": 5, "token": -1}
 
 
 def run_profile_kernel(args):
@@ -330,6 +331,8 @@ def run_profile_kernel(args):
         i4.set_option("gemv_ctas_per_sm", args.gemv_ctas)
     if args.l2_prefetch is not None:
         i4.set_option("l2_prefetch", args.l2_prefetch)
+    if args.persistent is not None:
+        i4.set_option("persistent", args.persistent)
     shape = synth.ModelShape(layers=1)
     dev = torch.device("cuda", 0)
     layers = [synth.layer_weights(synth.QWEN7B, 0, 0)]
@@ -340,12 +343,68 @@ def run_profile_kernel(args):
     for _ in range(args.prime_steps):
         graph.replay()
     k = PROFILE_KERNELS[args.profile_kernel]
-    index = k if k < 5 else graph.kernel_count - 1
+    index = k if k < 5 else graph.phase_count - 1
     for _ in range(args.launches):
-        graph.launch_kernel(index)
+        if k < 0:
+            graph.replay()  # the whole one-layer token step
+        else:
+            graph.launch_kernel(index)
     torch.cuda.synchronize()
     print(json.dumps({"profile_kernel": args.profile_kernel, "index": index, "launches": args.launches,
-                      "device_error": i4.device_error()}))
+                      "persistent": graph.persistent, "device_error": i4.device_error()}))
+    graph.close()
+    return 0
+
+
+def run_trace_step(args):
+    """Phase timestamps of one persistent decode step of the 7B-shape model after a --prompt token prompt:
+    per phase kind, the median over CTAs of the time from the phase start (grid barrier passed) to its input
+    staged, from staged to done, and the barrier wait (the next phase's start after this CTA's done), in us;
+    the raw [phase][cta][4] array goes to the .npz path given."""
+    import numpy as np
+    import torch
+
+    import int4_weight_only_02_b200 as i4
+    from int4_weight_only_02_b200 import synth
+    dev = torch.device("cuda", 0)
+    i4.set_option("trace", 1)
+    if args.l2_ahead is not None:
+        i4.set_option("l2_ahead", args.l2_ahead)
+    shape = synth.QWEN7B
+    model = i4.DeviceModel.synthetic(shape, device=dev)
+    seq = i4.Sequence(model, synth.page_table(shape, 0), synth.prompt_tokens(shape, args.prompt, 0))
+    graph = i4.DecodeGraph(model, seq)
+    if not graph.persistent:
+        raise SystemExit("the trace needs the persistent step")
+    for _ in range(args.prompt + 2):
+        graph.replay()
+    torch.cuda.synchronize()
+    grid = torch.cuda.get_device_properties(dev).multi_processor_count
+    tr = graph.trace(grid).astype(np.int64)
+    np.savez(args.trace_step, trace=tr)
+    kinds = ["qkv", "attention", "o", "gate_up", "down"]
+    t0 = tr[0, :, 0].min()
+    out = {}
+    for pi in range(tr.shape[0]):
+        kind = "lm_head" if pi == tr.shape[0] - 1 else kinds[pi % 5]
+        start, staged, done = tr[pi, :, 0], tr[pi, :, 1], tr[pi, :, 2]
+        nxt = tr[pi + 1, :, 0] if pi + 1 < tr.shape[0] else None
+        has = done > 0
+        rec = out.setdefault(kind, {"stage_us": [], "work_us": [], "wait_us": [], "span_us": []})
+        if kind != "attention":
+            m = has & (staged > 0)
+            rec["stage_us"].append(float(np.median(staged[m] - start[m])) / 1e3 if m.any() else 0.0)
+            rec["work_us"].append(float(np.median(done[m] - staged[m])) / 1e3 if m.any() else 0.0)
+        else:
+            rec["work_us"].append(float(np.median(done - start)) / 1e3)
+        if nxt is not None:
+            m = has
+            rec["wait_us"].append(float(np.median(nxt[m] - done[m])) / 1e3 if m.any() else 0.0)
+            rec["span_us"].append(float(nxt.min() - start.min()) / 1e3)
+    summary = {k: {kk: round(float(np.mean(v)), 3) for kk, v in r.items() if v} for k, r in out.items()}
+    print(json.dumps({"trace_step": args.trace_step, "ctx": int(seq.ctx_len.item()),
+                      "token_us": round(float(tr[-1, :, 2].max() - t0) / 1e3, 1), "per_phase_mean": summary,
+                      "device_error": i4.device_error()}), flush=True)
     graph.close()
     return 0
 
@@ -592,11 +651,17 @@ def main():
     ap.add_argument("--unpack", type=int, default=None, help="override the GEMV unpack variant (0..4, 4 = per shape)")
     ap.add_argument("--gemv-ctas", type=int, default=None, help="override the GEMV CTAs per SM (1 or 2)")
     ap.add_argument("--l2-prefetch", type=int, default=None, help="override the next-GEMV L2 prefetch (0/1)")
+    ap.add_argument("--l2-ahead", type=int, default=None,
+                    help="override the tiles each CTA of the persistent step prefetches into L2 ahead (0..64)")
+    ap.add_argument("--persistent", type=int, default=None,
+                    help="override the persistent one-kernel step (1) against one kernel per phase (0)")
     ap.add_argument("--profile-kernel", default=None, choices=sorted(PROFILE_KERNELS),
                     help="profiling mode: a one-layer model of the same shapes, then only this kernel of the "
                          "decode step, --launches times (for ncu captures)")
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--prime-steps", type=int, default=0, help="profiling mode: decode steps run first")
+    ap.add_argument("--trace-step", default=None,
+                    help="phase timestamps of one persistent decode step, raw array saved to this .npz path")
     ap.add_argument("--attention-sweep", action="store_true",
                     help="paged attention sweep over contexts, page sizes 16/64 and batches 1/8/32 (KV GB/s)")
     ap.add_argument("--sweep-contexts", default="512,2048,8192,32768")
@@ -611,6 +676,8 @@ def main():
         return run_reference(args)
     if args.profile_kernel:
         return run_profile_kernel(args)
+    if args.trace_step:
+        return run_trace_step(args)
     if args.attention_sweep:
         return run_attention_sweep(args)
     if args.gemv_batch:
@@ -647,6 +714,10 @@ def main():
         i4.set_option("gemv_ctas_per_sm", args.gemv_ctas)
     if args.l2_prefetch is not None:
         i4.set_option("l2_prefetch", args.l2_prefetch)
+    if args.persistent is not None:
+        i4.set_option("persistent", args.persistent)
+    if args.l2_ahead is not None:
+        i4.set_option("l2_ahead", args.l2_ahead)
 
     shape = synth.QWEN7B
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
@@ -768,19 +839,33 @@ def main():
     # lm_head: the last kernel of the step, launched 28 times (it also advances the sequence state,
     # which nothing reads afterwards)
     lm_bytes = shape.vocab * (h // 2) + shape.vocab * (h // 128) * 2 + shape.vocab * 4 + 2 * h * 2
-    lm_ms = time_kernel(lambda li: n_k - 1)
+    lm_ms = time_kernel(lambda li: graph.phase_count - 1)
     torch.cuda.synchronize()
     # restore a consistent residual/KV state is not needed afterwards: nothing else runs
 
     peak, peak_kind = measured_peaks()
     gu_gbs = gu_bytes / (gu_ms * 1e-3) / 1e9
-    traffic = traffic_from_profile("gemv_gate_up_qwen7b.md", GEMV_SOURCES)
 
     weight_bytes = model.weight_bytes()
     ctx_mean = (ctx0 + ctx1 - 1) / 2.0
     kv_bytes = 2 * shape.layers * shape.n_kv * shape.head_dim * 2 * ctx_mean
     step_bytes = weight_bytes + kv_bytes
     step_gbs = step_bytes / (ms_tok * 1e-3) / 1e9
+    if graph.persistent:
+        # the dominant (and only) kernel: one launch per token streams every weight byte and the context's K/V
+        roofline = {"kernel": "decode_persistent_kernel: the whole token (28 x {qkv, attention, o, gate/up, "
+                              "down} + lm_head) in one launch, one CTA per SM",
+                    "bound": "hbm", "achieved": round(step_gbs, 1), "peak": peak,
+                    "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s", "frac": round(step_gbs / peak, 4),
+                    "traffic": traffic_from_profile("decode_persistent_qwen7b.md", PERSIST_SOURCES),
+                    "bytes_per_launch": int(step_bytes), "us_per_launch": round(ms_tok * 1e3, 2),
+                    "timing": "CUDA events over the timed graph replays (one kernel per replay)"}
+    else:
+        roofline = {"kernel": "rmsnorm+gate/up int4 gemv+silu (K=3584, N=37888)", "bound": "hbm",
+                    "achieved": round(gu_gbs, 1), "peak": peak, "peak_kind": f"{peak_kind} copy bandwidth",
+                    "unit": "GB/s", "frac": round(gu_gbs / peak, 4),
+                    "traffic": traffic_from_profile("gemv_gate_up_qwen7b.md", GEMV_SOURCES),
+                    "bytes_per_launch": gu_bytes, "us_per_launch": round(gu_ms * 1e3, 2)}
 
     line = {
         "metric": METRIC, "value": round(job_tokens_per_s(args.steps, world, ms_max), 2), "unit": "tok/s",
@@ -791,11 +876,10 @@ def main():
                    "arith": "int4 weights x fp16 activations, fp32 accumulate", "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2: 3.65 GB of weights streamed per step, no flush",
                    "kernels_per_step": n_k, "status": status},
-        "roofline": {"kernel": "rmsnorm+gate/up int4 gemv+silu (K=3584, N=37888)", "bound": "hbm",
-                     "achieved": round(gu_gbs, 1), "peak": peak, "peak_kind": f"{peak_kind} copy bandwidth",
-                     "unit": "GB/s", "frac": round(gu_gbs / peak, 4), "traffic": traffic,
-                     "bytes_per_launch": gu_bytes, "us_per_launch": round(gu_ms * 1e3, 2)},
-        "kernels": {
+        "roofline": roofline,
+        "persistent_step": graph.persistent,
+        # each phase launched alone (its own launch, stream start-up and drain): diagnostics only
+        "phase_launches": {
             "qkv": {"us": round(qkv_ms * 1e3, 2), "GBs": round(qkv_bytes / (qkv_ms * 1e-3) / 1e9, 1)},
             "o": {"us": round(o_ms * 1e3, 2), "GBs": round(o_bytes / (o_ms * 1e-3) / 1e9, 1)},
             "gate_up": {"us": round(gu_ms * 1e3, 2), "GBs": round(gu_gbs, 1)},

@@ -278,17 +278,51 @@ I4_API int decode_step_graph_create(const i4_model_desc *desc, const i4_model_we
 I4_API int decode_step_graph_replay(i4_graph *g, void *stream);
 /* The same step as individual kernel launches on `stream` (no graph). */
 I4_API int decode_step_eager(i4_graph *g, void *stream);
-/* Kernel launches in one step (eager or inside the graph). */
+/* Kernel launches in one step (eager or inside the graph): 1 for the persistent
+ * step, 5 * n_layers + 1 for the per-kernel step. */
 I4_API int decode_step_kernel_count(const i4_graph *g);
+/* Phases of one step: 5 * n_layers + 1 (per layer qkv, attention, o, gate/up,
+ * down; then lm_head). */
+I4_API int decode_step_phase_count(const i4_graph *g);
+/* 1 when the step runs as one persistent kernel, 0 for one kernel per phase. */
+I4_API int decode_step_is_persistent(const i4_graph *g);
+/*
+ * Diagnostics of a persistent step created with the "trace" option: copies the
+ * timestamps (GPU global timer, ns) of the last launch to HOST memory
+ * `host_out` of n >= phase_count * grid * 4 entries, laid out [phase][cta][4]:
+ * consumers begin the phase, its input vector is staged, its work is done, and
+ * the producer issues the phase's first tile (0 where the CTA had no such
+ * event); for attention phases entries 1 and 3 are the CTA's key tiles done
+ * and its partial result published. Synchronous.
+ */
+I4_API int decode_step_trace(i4_graph *g, unsigned long long *host_out, size_t n);
 I4_API int decode_step_graph_destroy(i4_graph *g);
 /*
- * Benchmark export: launch only kernel `index` (0 <= index < kernel count) of
- * the step on `stream`, with the step's arguments. Per layer l the kernels are
- * 5l+0 qkv, 5l+1 attention, 5l+2 o, 5l+3 gate/up, 5l+4 down; the last is
- * lm_head + argmax, which advances the sequence state. Kernels that add into
- * the residual or write K/V leave values that the next full step rewrites.
+ * Test and benchmark export: run only phase `index` (0 <= index < phase count)
+ * of the step on `stream`, with the step's arguments, as one launch. Per layer
+ * l the phases are 5l+0 qkv, 5l+1 attention, 5l+2 o, 5l+3 gate/up, 5l+4 down;
+ * the last is lm_head + argmax, which advances the sequence state. Phases that
+ * add into the residual or write K/V leave values that the next full step
+ * rewrites.
  */
 I4_API int decode_step_launch_kernel(i4_graph *g, int index, void *stream);
+
+/*
+ * Test export: copy one of the step's own activation buffers to (dir = 0) or
+ * from (dir = 1) the caller's device buffer `dev`, asynchronously on `stream`.
+ * `bytes` must equal the buffer's size:
+ *   I4_BUF_RESID  the fp16 residual stream [hidden];
+ *   I4_BUF_Q      q after RoPE, fp16 [n_q_heads * head_dim];
+ *   I4_BUF_ATTN   the attention output, fp16 [n_q_heads * head_dim];
+ *   I4_BUF_MLP    SiLU(gate) * up, fp16 [intermediate].
+ * With decode_step_launch_kernel this lets a test give one kernel of the step
+ * chosen inputs and read back its outputs.
+ */
+#define I4_BUF_RESID 0
+#define I4_BUF_Q 1
+#define I4_BUF_ATTN 2
+#define I4_BUF_MLP 3
+I4_API int decode_step_buffer_copy(i4_graph *g, int which, void *dev, size_t bytes, int dir, void *stream);
 
 /*
  * Library options, applied to graphs created afterwards and to later calls:
@@ -306,6 +340,14 @@ I4_API int decode_step_launch_kernel(i4_graph *g, int index, void *stream);
  *            (M == 1, K % 512 == 0, 16-byte aligned w and scales), default 1;
  *   "stream_smem_kb" 32..227: shared memory budget of that kernel's ring;
  *   "gemv_ctas_per_sm" 1/2 (default 2): CTAs per SM of the pipelined GEMV grids;
+ *   "l2_ahead" 0..64 (default 8): tiles of its own weight stream each CTA of a
+ *            persistent step prefetches into L2 ahead of its shared-memory ring;
+ *   "trace"  0/1 (default 0): persistent steps created afterwards record phase
+ *            timestamps (see decode_step_trace);
+ *   "persistent" 0/1 (default 1): build decode steps as one persistent kernel
+ *            per token (one CTA per SM running every phase, the weight stream
+ *            never stopping at phase boundaries; shapes it does not cover fall
+ *            back to one kernel per phase);
  *   "l2_prefetch" 0/1 (default 0): in a decode step, each GEMV prefetches the
  *            next GEMV's weights into L2 (up to 48 MB) once its own ring is full.
  * Not thread-safe; set options before creating graphs.

@@ -83,8 +83,12 @@ _SIGS = {
     "decode_step_graph_replay": (_i, [_vp, _vp]),
     "decode_step_eager": (_i, [_vp, _vp]),
     "decode_step_kernel_count": (_i, [_vp]),
+    "decode_step_phase_count": (_i, [_vp]),
+    "decode_step_is_persistent": (_i, [_vp]),
+    "decode_step_trace": (_i, [_vp, ctypes.POINTER(ctypes.c_ulonglong), _sz]),
     "decode_step_graph_destroy": (_i, [_vp]),
     "decode_step_launch_kernel": (_i, [_vp, _i, _vp]),
+    "decode_step_buffer_copy": (_i, [_vp, _i, _vp, _sz, _i, _vp]),
     "i4_set_option": (_i, [ctypes.c_char_p, _i]),
     "i4_device_error": (_i, [_i]),
 }

@@ -38,6 +38,7 @@
 #include "async.cuh"
 #include "attention.cuh"
 #include "common.cuh"
+#include "mma.cuh"
 
 namespace i4 {
 
@@ -110,34 +111,6 @@ AttnWs attn_ws_layout(int B, int Hq, int Hkv, int page_size, int max_pages) {
 
 // ------------------------------------------------------------------ device helpers
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-
-// d += A(16x16, row) * B(16x8, col), fp16 inputs, fp32 accumulation
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -158,8 +131,6 @@ __device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, f
 __device__ __forceinline__ void st_cluster_f2(uint32_t addr, float a, float b) {
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
 }
-__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
-
 // oh[h] = sum_k cw[k][h] * part[k][d][h] over n <= N partials laid out [k][dim][head]
 template <int N>
 __device__ __forceinline__ void combine(float (&oh)[kMaxGroup], const float *part, const float (*cw)[kMaxGroup],
@@ -183,11 +154,6 @@ __device__ __forceinline__ void combine(float (&oh)[kMaxGroup], const float *par
             oh[7] = fmaf(wh.w, hi.w, oh[7]);
         }
     }
-}
-
-// weight of a partial with maximum m under the merged maximum M (0 for an empty partial)
-__device__ __forceinline__ float merge_weight(float m, float M) {
-    return m == -INFINITY ? 0.f : exp2f(m - (M == -INFINITY ? 0.f : M));
 }
 
 // ------------------------------------------------------------------ the kernel

@@ -24,6 +24,7 @@
 #include "attention.cuh"
 #include "common.cuh"
 #include "gemv.cuh"
+#include "persist.cuh"
 
 namespace i4 {
 int launch_rope_table(float2 *cs, int max_ctx, int d, double theta, cudaStream_t stream);
@@ -31,6 +32,9 @@ extern bool g_l2_prefetch;
 bool g_dry_run = false;
 bool g_pdl = true;
 bool g_l2_prefetch = false;
+bool g_persistent = false;
+bool g_trace = false;
+int g_l2_ahead = 8;
 }  // namespace i4
 
 using namespace i4;
@@ -55,9 +59,29 @@ struct i4_graph {
     bool l2pf = false;  // each GEMV prefetches the next GEMV's weights into L2
     int unpack = UNPACK_EXACT;
     int n_kernels = 0;
+    // persistent step: one kernel per token over all phases (persist.cu)
+    bool persistent = false;
+    bool coop = true;
+    PersistPlan plan = {};
+    PersistArgs pargs = {};
+    int n_phases = 0;
+    unsigned long long *trace = nullptr;  // [phase][cta][4] timestamps when created with the "trace" option
 };
 
+// Phases [begin, end) of the persistent step as one launch.
+static int launch_phases(i4_graph *g, cudaStream_t st, int begin, int end) {
+    if (g_dry_run) return persist_configure(g->plan);
+    PersistArgs a = g->pargs;
+    a.phase_begin = begin;
+    a.phase_end = end;
+    return persist_launch(a, g->plan, st, g->coop);
+}
+
 static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1) {
+    if (g->persistent) {
+        if (count) *count = 1;
+        return only >= 0 ? launch_phases(g, st, only, only + 1) : launch_phases(g, st, 0, g->n_phases);
+    }
     const i4_model_desc &d = g->d;
     const int H = d.hidden, I = d.intermediate, D = d.head_dim;
     const int nqkv = (d.n_q_heads + 2 * d.n_kv_heads) * D;
@@ -294,6 +318,13 @@ extern "C" int decode_step_graph_create(const i4_model_desc *desc, const i4_mode
     const size_t o_rope = off; off += a256((size_t)desc->max_ctx * (D / 2) * sizeof(float2));
     const size_t o_best = off; off += 256;
     const size_t o_attn_ws = off; off += a256(g->attn_layout.bytes);
+    g->n_phases = 5 * desc->n_layers + 1;
+    if (g_persistent) g->plan = persist_plan(*desc);
+    g->persistent = g_persistent && g->plan.ok;
+    const size_t o_phases = off; off += g->persistent ? a256(sizeof(PPhase) * g->n_phases) : 0;
+    const size_t o_pws = off; off += g->persistent ? a256(g->plan.ws_bytes) : 0;
+    const size_t trace_bytes = (size_t)g->n_phases * g->plan.grid * 4 * sizeof(unsigned long long);
+    const size_t o_trace = off; off += (g->persistent && g_trace) ? a256(trace_bytes) : 0;
     if (cudaMalloc(&g->ws, off) != cudaSuccess) {
         cudaGetLastError();
         release(g);
@@ -308,16 +339,82 @@ extern "C" int decode_step_graph_create(const i4_model_desc *desc, const i4_mode
     g->arrive = reinterpret_cast<unsigned *>(g->ws + o_best + 8);
     g->attn_ws = g->ws + o_attn_ws;
 
+    std::vector<PPhase> phases;
+    if (g->persistent) {
+        phases.resize(g->n_phases);
+        persist_fill_phases(*desc, g->plan, phases.data());
+        for (int i = 0; i < g->n_phases; ++i) {
+            PPhase &p = phases[i];
+            const i4_layer_weights *L = p.layer < desc->n_layers ? &g->layers[p.layer] : nullptr;
+            switch (p.kind) {
+                case PH_QKV: p.w = L->w_qkv; p.s = L->s_qkv; p.gamma = L->ln_in; p.bias = L->b_qkv;
+                             p.k_pool = g->kp[p.layer]; p.v_pool = g->vp[p.layer]; break;
+                case PH_ATTN: p.k_pool = g->kp[p.layer]; p.v_pool = g->vp[p.layer]; break;
+                case PH_O: p.w = L->w_o; p.s = L->s_o; break;
+                case PH_GU: p.w = L->w_gate_up; p.s = L->s_gate_up; p.gamma = L->ln_post; break;
+                case PH_DOWN: p.w = L->w_down; p.s = L->s_down; break;
+                case PH_LM: p.w = g->w.w_lm; p.s = g->w.s_lm; p.gamma = g->w.ln_final; break;
+            }
+        }
+        PersistArgs &a = g->pargs;
+        a.phases = reinterpret_cast<const PPhase *>(g->ws + o_phases);
+        a.slot_bytes = g->plan.slot_bytes;
+        a.stages = g->plan.stages;
+        a.l2_ahead = g_l2_ahead;
+        a.resid = g->resid;
+        a.q = g->q;
+        a.attn = g->attn;
+        a.mlp = g->mlp;
+        a.logits = seq->logits;
+        a.embed = weights->embed;
+        a.rope_cs = g->rope_cs;
+        a.vocab = desc->vocab;
+        a.hidden = H;
+        a.inter = desc->intermediate;
+        a.n_q = desc->n_q_heads;
+        a.n_kv = desc->n_kv_heads;
+        a.page_size = desc->page_size;
+        a.max_pages = pages;
+        a.max_ctx = desc->max_ctx;
+        a.eps = desc->rms_eps;
+        a.attn_scale = (float)(1.0 / std::sqrt((double)D));
+        a.token = seq->token;
+        a.pos = seq->pos;
+        a.ctx_len = seq->ctx_len;
+        a.status = seq->status;
+        a.history = seq->history;
+        a.prompt = seq->prompt;
+        a.n_prompt = seq->prompt ? seq->n_prompt : 0;
+        a.page_table = seq->page_table;
+        char *pw = g->ws + o_pws;
+        a.bar_count = reinterpret_cast<unsigned long long *>(pw);
+        a.best = reinterpret_cast<unsigned long long *>(pw + 8);
+        a.arrive = reinterpret_cast<unsigned *>(pw + 16);
+        a.attn_count = reinterpret_cast<unsigned *>(pw + 256);
+        a.attn_max_splits = g->plan.attn_max_splits;
+        const size_t cells = (size_t)desc->n_kv_heads * g->plan.attn_max_splits * 8;
+        a.attn_ml = reinterpret_cast<float2 *>(pw + 512);
+        a.attn_acc = reinterpret_cast<float *>(pw + 512 + a256(cells * sizeof(float2)));
+        if (g_trace) g->trace = a.trace = reinterpret_cast<unsigned long long *>(g->ws + o_trace);
+    }
     if ((st = cuda_check(cudaStreamCreateWithFlags(&g->cap, cudaStreamNonBlocking), "stream create")) ||
         (st = cuda_check(cudaMemsetAsync(g->ws, 0, off, g->cap), "workspace clear")) ||
         (st = launch_rope_table(g->rope_cs, desc->max_ctx, D, (double)desc->rope_theta, g->cap)) ||
+        (g->persistent &&
+         (st = cuda_check(cudaMemcpyAsync(g->ws + o_phases, phases.data(), sizeof(PPhase) * g->n_phases,
+                                          cudaMemcpyHostToDevice, g->cap), "phase table upload"))) ||
         (st = cuda_check(cudaStreamSynchronize(g->cap), "workspace init"))) {
         release(g);
         return st;
     }
-    // configure every kernel variant (shared-memory limits, occupancy) outside the capture
+    // configure every kernel variant (shared-memory limits, occupancy) outside the capture; a persistent
+    // step the device cannot hold (one CTA per SM) falls back to one kernel per phase
     g_dry_run = true;
     st = enqueue_step(g, g->cap, &g->n_kernels);
+    if (st && g->persistent) {
+        g->persistent = false;
+        st = enqueue_step(g, g->cap, &g->n_kernels);
+    }
     g_dry_run = false;
     if (st) {
         release(g);
@@ -352,11 +449,43 @@ extern "C" int decode_step_eager(i4_graph *g, void *stream) {
 
 extern "C" int decode_step_kernel_count(const i4_graph *g) { return g ? g->n_kernels : 0; }
 
+extern "C" int decode_step_phase_count(const i4_graph *g) { return g ? g->n_phases : 0; }
+
 extern "C" int decode_step_launch_kernel(i4_graph *g, int index, void *stream) {
     if (!g) return fail(I4_EINVAL, "decode_step_launch_kernel: no graph");
-    if (index < 0 || index >= g->n_kernels)
-        return fail(I4_EINVAL, "decode_step_launch_kernel: index %d outside [0, %d)", index, g->n_kernels);
+    if (index < 0 || index >= g->n_phases)
+        return fail(I4_EINVAL, "decode_step_launch_kernel: index %d outside [0, %d)", index, g->n_phases);
     return enqueue_step(g, (cudaStream_t)stream, nullptr, index);
+}
+
+extern "C" int decode_step_is_persistent(const i4_graph *g) { return g && g->persistent ? 1 : 0; }
+
+extern "C" int decode_step_trace(i4_graph *g, unsigned long long *host_out, size_t n) {
+    if (!g || !host_out) return fail(I4_EINVAL, "decode_step_trace: null argument");
+    if (!g->trace) return fail(I4_EINVAL, "decode_step_trace: graph was not created with the \"trace\" option");
+    const size_t need = (size_t)g->n_phases * g->plan.grid * 4;
+    if (n < need) return fail(I4_EINVAL, "decode_step_trace: %zu entries needed", need);
+    return cuda_check(cudaMemcpy(host_out, g->trace, need * sizeof(unsigned long long), cudaMemcpyDeviceToHost),
+                      "decode_step_trace");
+}
+
+extern "C" int decode_step_buffer_copy(i4_graph *g, int which, void *dev, size_t bytes, int dir, void *stream) {
+    if (!g || !dev) return fail(I4_EINVAL, "decode_step_buffer_copy: null argument");
+    if (dir != 0 && dir != 1) return fail(I4_EINVAL, "decode_step_buffer_copy: dir must be 0 (out) or 1 (in)");
+    uint16_t *buf = nullptr;
+    size_t n = 0;
+    switch (which) {
+        case I4_BUF_RESID: buf = g->resid; n = (size_t)g->d.hidden * 2; break;
+        case I4_BUF_Q: buf = g->q; n = (size_t)g->d.n_q_heads * g->d.head_dim * 2; break;
+        case I4_BUF_ATTN: buf = g->attn; n = (size_t)g->d.n_q_heads * g->d.head_dim * 2; break;
+        case I4_BUF_MLP: buf = g->mlp; n = (size_t)g->d.intermediate * 2; break;
+        default: return fail(I4_EINVAL, "decode_step_buffer_copy: unknown buffer %d", which);
+    }
+    if (bytes != n) return fail(I4_EINVAL, "decode_step_buffer_copy: buffer %d holds %zu bytes, got %zu", which, n, bytes);
+    void *dst = dir == 0 ? dev : (void *)buf;
+    const void *src = dir == 0 ? (const void *)buf : dev;
+    return cuda_check(cudaMemcpyAsync(dst, src, n, cudaMemcpyDeviceToDevice, (cudaStream_t)stream),
+                      "decode_step_buffer_copy");
 }
 
 extern "C" int decode_step_graph_destroy(i4_graph *g) {
@@ -382,6 +511,19 @@ extern "C" int i4_set_option(const char *name, int value) {
     }
     if (n == "stream") {
         set_stream_options(value, 0);
+        return I4_OK;
+    }
+    if (n == "l2_ahead") {
+        if (value < 0 || value > 64) return fail(I4_EINVAL, "l2_ahead must be in [0, 64]");
+        g_l2_ahead = value;
+        return I4_OK;
+    }
+    if (n == "trace") {
+        g_trace = value != 0;
+        return I4_OK;
+    }
+    if (n == "persistent") {
+        g_persistent = value != 0;
         return I4_OK;
     }
     if (n == "l2_prefetch") {

@@ -5,6 +5,7 @@
 
 #include "common.cuh"
 #include "gemv.cuh"
+#include "mma.cuh"
 
 namespace i4 {
 
@@ -618,6 +619,97 @@ __device__ __forceinline__ void finish_step(const GemvArgs &a, unsigned long lon
     *a.best = 0ull;
     *a.arrive = 0u;
     __threadfence();
+}
+
+// ---------------------------------------------------------------- tensor-core row-pair dot product
+
+// One 1024-weight block of the row pair (a, b) on tensor cores: lane (g, c)
+// holds 16 contiguous bytes of each row (32 weights, all in group 8b + g),
+// unpacked with one shift and four LOP3s per word into offset-binary fp16
+// subnormals (u * 2^-24 for low fields, 16u * 2^-24 for high fields) as the A
+// operand of mma.m16n8k16; its B fragment is x at the same k. B column g is fed
+// only by lanes (g, *), so D[g][g] is row a's dot product over the lane group's
+// 128-weight group and D[g + 8][g] row b's; lane (g, g / 2) holds both and adds
+// s * ((lo + hi / 16) * 2^24 - 8 * sum(x)) to tot. Other lanes add garbage that
+// the caller never reads (it masks them before the warp sum).
+__device__ __forceinline__ void block_dot(uint4 qa, uint4 qb, const uint4 *xb, float sxj, float sa, float sb,
+                                          bool odd, float2 &tot) {
+    const uint32_t wra[4] = {qa.x, qa.y, qa.z, qa.w}, wrb[4] = {qb.x, qb.y, qb.z, qb.w};
+    float lo[4], hi[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint4 xc = xb[w * 32];  // (x0,x4) (x2,x6) (x1,x5) (x3,x7)
+        uint32_t ua[4], ub[4];
+        unpack_word_subnormal(wra[w], ua);  // (k0,k4) 16(k1,k5) (k2,k6) 16(k3,k7)
+        unpack_word_subnormal(wrb[w], ub);
+        if (w == 0) {
+            mma16816_z(lo, ua[0], ub[0], ua[2], ub[2], xc.x, xc.y);
+            mma16816_z(hi, ua[1], ub[1], ua[3], ub[3], xc.z, xc.w);
+        } else {
+            mma16816(lo, ua[0], ub[0], ua[2], ub[2], xc.x, xc.y);
+            mma16816(hi, ua[1], ub[1], ua[3], ub[3], xc.z, xc.w);
+        }
+    }
+    const float2 l2 = odd ? make_float2(lo[1], lo[3]) : make_float2(lo[0], lo[2]);
+    const float2 h2 = odd ? make_float2(hi[1], hi[3]) : make_float2(hi[0], hi[2]);
+    const float2 v = ffma2(ffma2(h2, make_float2(0.0625f, 0.0625f), l2), make_float2(16777216.0f, 16777216.0f),
+                           make_float2(-sxj, -sxj));
+    tot = ffma2(v, make_float2(sa, sb), tot);
+}
+
+// Row pair (slot rows row_a, row_b) against x over blocks [b0, b1); K is a
+// compile-time constant when KC > 0 (all offsets then become immediates).
+template <int KC>
+__device__ __forceinline__ float2 pair_dot(const unsigned char *st, int K, int row_a, int row_b, const uint16_t *sa,
+                                           const uint16_t *sb, const uint4 *xt, const float *sx8, int b0, int b1,
+                                           int lane) {
+    const int Kk = KC ? KC : K, wrow = Kk >> 1, groups = Kk >> 7, kfull = Kk >> 10;
+    const int g = lane >> 2, c = lane & 3;
+    const bool diag = c == (g >> 1), odd = g & 1;
+    const unsigned char *wa = st + (size_t)row_a * wrow + 16 * lane;
+    const unsigned char *wb = st + (size_t)row_b * wrow + 16 * lane;
+    const uint4 *xl = xt + lane;
+    float2 tot = make_float2(0.f, 0.f);
+    auto full_block = [&](int b) {
+        const uint4 qa = *reinterpret_cast<const uint4 *>(wa + 512 * b);
+        const uint4 qb = *reinterpret_cast<const uint4 *>(wb + 512 * b);
+        const int j = 8 * b + g;
+        block_dot(qa, qb, xl + b * 128, sx8[j], half_bits_to_float(sa[j]), half_bits_to_float(sb[j]), odd, tot);
+    };
+    auto part_block = [&](int b) {  // past K: all-zero codes (u = 0); groups past K are never read
+        uint4 qa = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u), qb = qa;
+        if (1024 * b + 32 * lane < Kk) {
+            qa = *reinterpret_cast<const uint4 *>(wa + 512 * b);
+            qb = *reinterpret_cast<const uint4 *>(wb + 512 * b);
+        }
+        // lanes of groups past K hold zero codes; their scales and sums are zero too, so they add nothing
+        const int j = 8 * b + g;
+        const bool in = j < groups;
+        block_dot(qa, qb, xl + b * 128, in ? sx8[j] : 0.f, in ? half_bits_to_float(sa[j]) : 0.f,
+                  in ? half_bits_to_float(sb[j]) : 0.f, odd, tot);
+    };
+    if constexpr (KC > 0) {
+        if (b0 == 0 && b1 == (KC + 1023) / 1024) {  // the whole row, unrolled
+#pragma unroll
+            for (int b = 0; b < KC / 1024; ++b) full_block(b);
+            if constexpr (KC % 1024) part_block(KC / 1024);
+            return diag ? tot : make_float2(0.f, 0.f);
+        }
+    }
+    const int bf = b1 < kfull ? b1 : kfull;
+#pragma unroll 2
+    for (int b = b0; b < bf; ++b) full_block(b);
+    for (int b = bf > b0 ? bf : b0; b < b1; ++b) part_block(b);
+    return diag ? tot : make_float2(0.f, 0.f);
+}
+
+__device__ __forceinline__ float2 warp_sum2(float2 v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+        v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
+    }
+    return v;
 }
 
 }  // namespace i4

@@ -341,7 +341,7 @@ __device__ __forceinline__ void stage_x_tc(const GemvArgs &a, uint4 *xt, float *
     }
 }
 
-template <int PRO, int EPI, int R>
+template <int PRO, int EPI, int R, int KC>
 __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvArgs a, const StreamGeom geo) {
     constexpr int PP = R / 2;               // row pairs per tile
     constexpr int WP = kConsumerWarps / PP;  // warps per row pair
@@ -396,8 +396,6 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvAr
         grp.sync();
         grid_dep_launch();
         const int c_id = grp.tid(), warp = c_id >> 5, lane = c_id & 31;
-        const int g = lane >> 2, c = lane & 3;
-        const bool diag = c == (g >> 1);  // this lane holds D[g][g] and D[g+8][g]
         const int pr = warp / WP, wp = warp % WP;
         const int b0 = (wp * nb) / WP, b1 = ((wp + 1) * nb) / WP;
         const int tra = kPaired<EPI> ? pr : 2 * pr, trb = kPaired<EPI> ? pr + PP : 2 * pr + 1;
@@ -421,56 +419,10 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvAr
             float tot_a = 0.f, tot_b = 0.f;
             if (live) {
                 const unsigned char *st = ring + (size_t)s * geo.stage_bytes;
-                const unsigned char *wa = st + (size_t)tra * wrow + 16 * lane;
-                const unsigned char *wb = st + (size_t)trb * wrow + 16 * lane;
                 const uint16_t *sa = reinterpret_cast<const uint16_t *>(st + (size_t)R * wrow) + tra * groups;
                 const uint16_t *sb = reinterpret_cast<const uint16_t *>(st + (size_t)R * wrow) + trb * groups;
-                float2 tot = make_float2(0.f, 0.f);  // rows (r, r')
-                // one block: the lane's 32 weights of each row, 8 MMAs, then this lane's group if it holds D[g][g]
-                auto block = [&](int b, auto partial) {
-                    uint4 qa, qb;
-                    if constexpr (decltype(partial)::value) {  // past K: all-zero codes (u = 0)
-                        qa = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
-                        qb = qa;
-                        if (1024 * b + 32 * lane < K) {
-                            qa = *reinterpret_cast<const uint4 *>(wa + 512 * b);
-                            qb = *reinterpret_cast<const uint4 *>(wb + 512 * b);
-                        }
-                    } else {
-                        qa = *reinterpret_cast<const uint4 *>(wa + 512 * b);
-                        qb = *reinterpret_cast<const uint4 *>(wb + 512 * b);
-                    }
-                    const uint32_t wra[4] = {qa.x, qa.y, qa.z, qa.w}, wrb[4] = {qb.x, qb.y, qb.z, qb.w};
-                    float lo[4], hi[4];
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const uint4 xc = xt[(b * 4 + w) * 32 + lane];  // (x0,x4) (x2,x6) (x1,x5) (x3,x7)
-                        uint32_t ua[4], ub[4];
-                        unpack_word_subnormal(wra[w], ua);  // (k0,k4) 16(k1,k5) (k2,k6) 16(k3,k7)
-                        unpack_word_subnormal(wrb[w], ub);
-                        if (w == 0) {  // first MMA of the block: accumulate onto zero
-                            mma_16816_z(lo, ua[0], ub[0], ua[2], ub[2], xc.x, xc.y);
-                            mma_16816_z(hi, ua[1], ub[1], ua[3], ub[3], xc.z, xc.w);
-                        } else {
-                            mma_16816(lo, ua[0], ub[0], ua[2], ub[2], xc.x, xc.y);
-                            mma_16816(hi, ua[1], ub[1], ua[3], ub[3], xc.z, xc.w);
-                        }
-                    }
-                    const int j = 8 * b + g;  // this lane's group
-                    if (diag && (!decltype(partial)::value || j < groups)) {
-                        const bool odd = g & 1;
-                        const float2 l2 = odd ? make_float2(lo[1], lo[3]) : make_float2(lo[0], lo[2]);
-                        const float2 h2 = odd ? make_float2(hi[1], hi[3]) : make_float2(hi[0], hi[2]);
-                        const float sxj = sx8[j];
-                        const float2 v = ffma2(ffma2(h2, make_float2(0.0625f, 0.0625f), l2),
-                                               make_float2(16777216.0f, 16777216.0f), make_float2(-sxj, -sxj));
-                        tot = ffma2(v, make_float2(half_bits_to_float(sa[j]), half_bits_to_float(sb[j])), tot);
-                    }
-                };
-                const int b_full = b1 < (K >> 10) ? b1 : (K >> 10);
-#pragma unroll 2
-                for (int b = b0; b < b_full; ++b) block(b, std::false_type{});
-                for (int b = b_full > b0 ? b_full : b0; b < b1; ++b) block(b, std::true_type{});
+                // K is a compile-time constant for the 7B shapes (KC > 0): offsets become immediates
+                const float2 tot = pair_dot<KC>(st, K, tra, trb, sa, sb, xt, sx8, b0, b1, lane);
                 tot_a = tot.x;
                 tot_b = tot.y;
             }
@@ -767,9 +719,9 @@ static int launch_stream_r(const GemvArgs &a, const StreamGeom &geo, cudaStream_
     }
 }
 
-template <int PRO, int EPI, int R>
-static int launch_tc_t(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
-    auto kern = gemv_tc_kernel<PRO, EPI, R>;
+template <int PRO, int EPI, int R, int KC>
+static int launch_tc_k(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
+    auto kern = gemv_tc_kernel<PRO, EPI, R, KC>;
     static int configured = -1;
     if (geo.smem > configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, geo.smem);
@@ -779,6 +731,18 @@ static int launch_tc_t(const GemvArgs &a, const StreamGeom &geo, cudaStream_t st
     if (g_dry_run) return I4_OK;
     return cuda_check(launch(kern, dim3(geo.grid), dim3(kStreamThreads), (size_t)geo.smem, stream, pdl, a, geo),
                       "tensor-core gemv launch");
+}
+
+// rows of 3584 weights (16-row tiles) and 18944 weights (2-row tiles), the decoder's two row lengths, get
+// kernels with K fixed at compile time; other shapes the generic one
+template <int PRO, int EPI, int R>
+static int launch_tc_t(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
+    if constexpr (R == 16) {
+        if (a.K == 3584) return launch_tc_k<PRO, EPI, R, 3584>(a, geo, stream, pdl);
+    } else {
+        if (a.K == 18944) return launch_tc_k<PRO, EPI, R, 18944>(a, geo, stream, pdl);
+    }
+    return launch_tc_k<PRO, EPI, R, 0>(a, geo, stream, pdl);
 }
 
 template <int EPI>
@@ -849,6 +813,7 @@ int read_gemv_error(int reset) {
 }
 
 int read_attn_error(int reset);
+int read_persist_error(int reset);
 
 }  // namespace i4
 
@@ -856,7 +821,9 @@ int read_attn_error(int reset);
 extern "C" int i4_device_error(int reset) {
     const int a = i4::read_gemv_error(reset);
     const int b = i4::read_attn_error(reset);
+    const int c = i4::read_persist_error(reset);
     if (a < 0) return a;
     if (b < 0) return b;
-    return a ? a : b;
+    if (c < 0) return c;
+    return a ? a : (b ? b : c);
 }

@@ -127,7 +127,24 @@ class DecodeGraph:
 
     @property
     def kernel_count(self) -> int:
+        """Kernel launches per step (1 for the persistent step)."""
         return int(lib().decode_step_kernel_count(self._h))
+
+    @property
+    def phase_count(self) -> int:
+        """Phases per step: 5 per layer (qkv, attention, o, gate/up, down) and lm_head."""
+        return int(lib().decode_step_phase_count(self._h))
+
+    @property
+    def persistent(self) -> bool:
+        return bool(lib().decode_step_is_persistent(self._h))
+
+    def trace(self, grid: int):
+        """Phase timestamps of the last launch [phase][cta][4] (ns; graphs created with the "trace" option)."""
+        n = self.phase_count * grid * 4
+        buf = (ctypes.c_ulonglong * n)()
+        _check(lib().decode_step_trace(self._h, buf, n), "decode_step_trace")
+        return np.frombuffer(buf, dtype=np.uint64).reshape(self.phase_count, grid, 4).copy()
 
     def replay(self, stream=None):
         _check(lib().decode_step_graph_replay(self._h, _stream(stream)), "decode_step_graph_replay")
@@ -136,7 +153,7 @@ class DecodeGraph:
         _check(lib().decode_step_eager(self._h, _stream(stream)), "decode_step_eager")
 
     def launch_kernel(self, index: int, stream=None):
-        """Launch only kernel `index` of the step (benchmarking; see decode_step_launch_kernel)."""
+        """Run only phase `index` of the step as one launch (tests, benchmarking; see decode_step_launch_kernel)."""
         _check(lib().decode_step_launch_kernel(self._h, index, _stream(stream)), "decode_step_launch_kernel")
 
     BUFFERS = {"resid": 0, "q": 1, "attn": 2, "mlp": 3}

@@ -73,11 +73,11 @@ def test_embed_gather_and_argmax_rows(i4lib, cuda):
     assert pos.cpu().tolist() == [1, 2, 3, 4] and ctx.cpu().tolist() == [2, 3, 4, 5]
 
 
-@pytest.mark.parametrize("inter,n_prompt,graph", [(1024, 24, True), (1024, 40, False), (4608, 40, True)])
+@pytest.mark.parametrize("inter,n_prompt,graph", [(1024, 24, True), (1024, 40, False), (12288, 40, True)])
 def test_chunked_prefill_matches_oracle(i4lib, cuda, inter, n_prompt, graph):
     """Prefill of one sequence 8 positions per step (rows = consecutive positions over one page-table
     row): the first generated token and the last position's logits equal the oracle's. Prompts of 3
-    and 5 chunks cross partially filled pages; eager and graph steps; intermediate 4608 sends the
+    and 5 chunks cross partially filled pages; eager and graph steps; intermediate 12288 sends the
     down projection through the split 4-vector calls."""
     import torch
     shape = synth.ModelShape(layers=2, hidden=512, inter=inter, n_q=4, n_kv=2, head_dim=128, vocab=1000,

@@ -30,7 +30,7 @@ MID = synth.ModelShape(layers=3, hidden=512, inter=1024, n_q=4, n_kv=1, head_dim
 LONG = synth.ModelShape(layers=2, hidden=512, inter=4608, n_q=4, n_kv=1, head_dim=128, vocab=2048, group=128,
                         page_size=16, max_ctx=256)
 SHAPES = {"small": SMALL, "mid": MID, "long": LONG}
-DEFAULT_UNPACK = 0
+DEFAULT_UNPACK = 4  # the library default: tensor-core kernels where they apply
 
 
 def small_setup(i4, cuda, seed=0, n_prompt=20, shape=SMALL):
@@ -47,9 +47,14 @@ def run_steps(graph, n, eager=False):
         graph.eager() if eager else graph.replay()
 
 
-@pytest.mark.parametrize("name,unpack", [("small", 0), ("mid", 0), ("mid", 1), ("mid", 2), ("mid", 3), ("long", 1),
-                                         ("long", 3)])
-def test_small_decoder_matches_oracle(i4lib, cuda, name, unpack):
+# (shape, unpack variant of the per-kernel step, persistent step); the small shape (rows of 256 and 384
+# weights) is outside the persistent step and always runs one kernel per phase
+CASES = [("small", 0, False), ("mid", 0, True), ("long", 0, True), ("mid", 0, False), ("mid", 1, False),
+         ("mid", 2, False), ("mid", 3, False), ("long", 1, False), ("long", 3, False)]
+
+
+@pytest.mark.parametrize("name,unpack,persistent", CASES)
+def test_small_decoder_matches_oracle(i4lib, cuda, name, unpack, persistent):
     import torch
     shape = SHAPES[name]
     layers, glob, table, prompt, model = small_setup(i4lib, cuda, shape=shape)
@@ -57,11 +62,15 @@ def test_small_decoder_matches_oracle(i4lib, cuda, name, unpack):
     ref_tokens, ref_logits = oracle.DecoderOracle(shape, layers, glob, table).generate(prompt, n_new)
     seq = i4lib.Sequence(model, table, prompt)
     i4lib.set_option("unpack", unpack)
+    i4lib.set_option("persistent", int(persistent))
     try:
         g = i4lib.DecodeGraph(model, seq)
     finally:
         i4lib.set_option("unpack", DEFAULT_UNPACK)
-    assert g.kernel_count == 5 * shape.layers + 1
+        i4lib.set_option("persistent", 1)
+    assert g.persistent == persistent
+    assert g.phase_count == 5 * shape.layers + 1
+    assert g.kernel_count == (1 if g.persistent else g.phase_count)
     logits = []
     for step in range(len(prompt) + n_new - 1):
         g.replay()
@@ -83,7 +92,7 @@ def test_small_decoder_matches_oracle(i4lib, cuda, name, unpack):
     g.close()
 
 
-@pytest.mark.parametrize("name", ["small", "mid"])
+@pytest.mark.parametrize("name", ["small", "mid", "long"])
 def test_graph_equals_eager_bit_exact(i4lib, cuda, name):
     import torch
     _, _, table, prompt, model = small_setup(i4lib, cuda, seed=1, n_prompt=9, shape=SHAPES[name])
@@ -102,15 +111,17 @@ def test_graph_equals_eager_bit_exact(i4lib, cuda, name):
         g.close()
 
 
-def test_context_limit_sets_status(i4lib, cuda):
+@pytest.mark.parametrize("name", ["small", "mid"])
+def test_context_limit_sets_status(i4lib, cuda, name):
     import torch
-    _, _, table, prompt, model = small_setup(i4lib, cuda, seed=2, n_prompt=4)
+    _, _, table, prompt, model = small_setup(i4lib, cuda, seed=2, n_prompt=4, shape=SHAPES[name])
     seq = i4lib.Sequence(model, table, prompt)
     g = i4lib.DecodeGraph(model, seq)
-    run_steps(g, SMALL.max_ctx + 3)
+    run_steps(g, SHAPES[name].max_ctx + 3)
     torch.cuda.synchronize()
     assert int(seq.status.item()) == 1
-    assert int(seq.pos.item()) == SMALL.max_ctx - 1
+    assert int(seq.pos.item()) == SHAPES[name].max_ctx - 1
+    assert i4lib.device_error() == 0
     g.close()
 
 
