@@ -65,13 +65,28 @@ I4_API const char *i4_version(void);
  *   scales [N][K/group] fp16, 2-byte aligned;
  *   x      [M][K] fp16, 16-byte aligned;  bias [N] fp16 or NULL;
  *   y      [M][N], 4-byte aligned for fp32.
- * Requires group == 128, K % 128 == 0, K <= 32768, 1 <= M <= 8, N >= 1; shapes
- * off the tensor-core paths stage the M vectors in shared memory, which allows
- * M <= 8 up to K = 12032 and M <= 4 up to K = 24064 (larger M * K is refused
- * with I4_EUNSUPPORTED). The kernel is chosen by the "unpack" option below.
+ * Requires group == 128, K % 128 == 0, K <= 32768, M >= 1, N >= 1. M > 8 runs
+ * int4_gemm below. For M <= 8, shapes off the tensor-core paths stage the M
+ * vectors in shared memory, which allows M <= 8 up to K = 12032 and M <= 4 up
+ * to K = 24064 (larger M * K is refused with I4_EUNSUPPORTED). The kernel is
+ * chosen by the "unpack" option below.
  */
 I4_API int int4_gemv(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
               int y_is_fp32, int M, int N, int K, int group, void *stream);
+
+/*
+ * The same INT4 linear layer for many activation rows (batched decode, prompt
+ * prefill) on the tcgen05 tensor cores: each 64-wide K chunk of 128 weight rows
+ * is dequantised to fp16 (q * s, rounded once) in shared memory and multiplied
+ * with the fp16 activations by tcgen05.mma into fp32 accumulators in tensor
+ * memory; y = accumulator (+ bias), stored as fp16 or fp32.
+ *   w [N][K/8] uint32 and x [M][K] fp16, 16-byte aligned; scales [N][K/128];
+ *   bias [N] or NULL; y [M][N]. group == 128, K % 128 == 0, K <= 65536.
+ * Any M >= 1 (tiles of 16 .. 512 activation rows per CTA); the tensor maps of
+ * w and x are encoded on the host at each call.
+ */
+I4_API int int4_gemm(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
+                     int y_is_fp32, int M, int N, int K, int group, void *stream);
 
 /*
  * Test export: q[n][k] = signed field of w (bit-exact unpack check).

@@ -64,6 +64,7 @@ _SIGS = {
     "i4_last_error": (ctypes.c_char_p, []),
     "i4_version": (ctypes.c_char_p, []),
     "int4_gemv": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "int4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "i4_int4_gemv_variant": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "i4_int4_unpack": (_i, [_vp, _vp, _i, _i, _vp]),
     "paged_gqa_decode_ws_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
@@ -160,6 +161,18 @@ def int4_gemv(w, scales, x, bias=None, y=None, out_fp32: bool = False, group: in
                                         0 if unpack is None else unpack, max_ctas, _stream(stream))
     _check(st, "int4_gemv")
     return y if x.dim() == 2 else y.view(-1)
+
+
+def int4_gemm(w, scales, x, bias=None, y=None, out_fp32: bool = False, group: int = 128, stream=None):
+    """y[M][N] = x[M][K] . dequant(w, scales)^T (+ bias) on the tcgen05 tensor cores (any M)."""
+    import torch
+    M, K = x.shape
+    N = w.shape[0]
+    if y is None:
+        y = torch.empty((M, N), device=x.device, dtype=torch.float32 if out_fp32 else torch.float16)
+    _check(lib().int4_gemm(_p(w), _p(scales), _p(x), _p(bias), _p(y), int(out_fp32), M, N, K, group,
+                           _stream(stream)), "int4_gemm")
+    return y
 
 
 def int4_unpack(w, K: int, stream=None):

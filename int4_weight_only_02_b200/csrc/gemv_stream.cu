@@ -814,6 +814,7 @@ int read_gemv_error(int reset) {
 
 int read_attn_error(int reset);
 int read_persist_error(int reset);
+int read_gemm_error(int reset);
 
 }  // namespace i4
 
@@ -822,8 +823,10 @@ extern "C" int i4_device_error(int reset) {
     const int a = i4::read_gemv_error(reset);
     const int b = i4::read_attn_error(reset);
     const int c = i4::read_persist_error(reset);
+    const int d = i4::read_gemm_error(reset);
     if (a < 0) return a;
     if (b < 0) return b;
     if (c < 0) return c;
-    return a ? a : (b ? b : c);
+    if (d < 0) return d;
+    return a ? a : (b ? b : (c ? c : d));
 }

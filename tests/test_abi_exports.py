@@ -19,7 +19,7 @@ def declared_symbols():
 
 def test_header_declares_the_boundary():
     names = declared_symbols()
-    for required in ["int4_gemv", "paged_gqa_decode", "paged_gqa_decode_ws_bytes", "rmsnorm_rope", "silu_mul",
+    for required in ["int4_gemv", "int4_gemm", "paged_gqa_decode", "paged_gqa_decode_ws_bytes", "rmsnorm_rope", "silu_mul",
                      "decode_step_graph_create", "decode_step_graph_replay", "decode_step_graph_destroy",
                      "decode_step_eager", "i4_int4_unpack", "i4_paged_gather", "i4_last_error"]:
         assert required in names
@@ -43,7 +43,12 @@ def test_host_validation_without_gpu(i4lib):
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
     assert L.int4_gemv(fake, fake, fake, None, fake, 0, 1, 16, 128, 64, None) == i4lib.I4_EUNSUPPORTED
     assert L.int4_gemv(fake, fake, fake, None, fake, 0, 1, 16, 100, 128, None) == i4lib.I4_EINVAL
-    assert L.int4_gemv(fake, fake, fake, None, fake, 0, 9, 16, 128, 128, None) == i4lib.I4_EUNSUPPORTED
+    # more than 8 rows go to the tcgen05 GEMM, which validates the same way before any launch
+    assert L.int4_gemv(fake, fake, fake, None, fake, 0, 9, 16, 128, 64, None) == i4lib.I4_EUNSUPPORTED
+    assert L.int4_gemm(fake, fake, fake, None, fake, 0, 512, 16, 100, 128, None) == i4lib.I4_EINVAL
+    assert L.int4_gemm(ctypes.c_void_p((1 << 20) + 8), fake, fake, None, fake, 0, 512, 16, 128, 128,
+                       None) == i4lib.I4_EALIGN
+    assert L.int4_gemm(None, fake, fake, None, fake, 0, 512, 16, 128, 128, None) == i4lib.I4_EINVAL
     odd = ctypes.c_void_p((1 << 20) + 4)
     assert L.int4_gemv(odd, fake, fake, None, fake, 0, 1, 16, 128, 128, None) == i4lib.I4_EALIGN
     assert L.paged_gqa_decode(fake, fake, fake, fake, fake, fake, 1, 28, 4, 64, 16, 4, 1.0, fake, 1 << 20,
