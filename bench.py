@@ -591,9 +591,12 @@ def run_batched_decode(args):
 
 
 def run_prefill(args):
-    """Time to first token of the 7B-shape decoder for a 512-token prompt, prefilled 8 positions per
-    step through the batched library calls (causal over one sequence's pages), against the same prompt
-    fed one token per step through the fused decode graph. One JSON line."""
+    """Time to first token of the 7B-shape decoder for a --prompt token prompt, every prompt position at once:
+    the linear layers on the tcgen05 INT4 GEMM (M = prompt rows), causal paged attention, lm_head for the last
+    position (Prefill.run, one stream, CUDA events around it after one warm-up run). Beside it: the same prompt
+    fed one token per step through the decode graph (the first tokens must agree), and one layer's parts at the
+    full prompt (each timed alone over 10 launches): the four GEMMs with their tensor throughput, attention and
+    the glue kernels. One JSON line; exit status 1 when the first tokens differ or a device error is set."""
     import numpy as np
     import torch
 
@@ -601,41 +604,90 @@ def run_prefill(args):
     from int4_weight_only_02_b200 import synth
     dev = torch.device("cuda", 0)
     shape = synth.QWEN7B
-    B = args.prefill
+    n = args.prompt
     model = i4.DeviceModel.synthetic(shape, device=dev)
     table = synth.page_table(shape, 0)
-    prompt = synth.prompt_tokens(shape, args.prompt, seed=0)
-    bd = i4.BatchedDecode(model, np.tile(table, (B, 1)), num_pages=shape.max_pages)
-    bd.prefill(prompt)  # warm-up (captures the step graph)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    prompt = synth.prompt_tokens(shape, n, seed=0)
+    seq = i4.Sequence(model, table, None)
+    pre = i4.Prefill(model, seq, max_tokens=n)
+    pre.run(prompt)  # warm-up: tensor maps, shared-memory attributes
     torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    tok = bd.prefill(prompt)
+    pre.run(prompt)
     e1.record()
     torch.cuda.synchronize()
-    chunked_ms = e0.elapsed_time(e1)
-    seq = i4.Sequence(model, table, prompt)
-    graph = i4.DecodeGraph(model, seq)
-    for _ in range(len(prompt)):
+    ttft_ms = e0.elapsed_time(e1)
+    tok = int(seq.token.item())
+
+    def timed(fn, reps=10):
+        fn()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    lw = model.layers[0]
+    h, inter, nqkv = shape.hidden, shape.inter, shape.qkv_rows
+    parts = {
+        "qkv_gemm": (lambda: i4.int4_gemm(lw["w_qkv"], lw["s_qkv"], pre.xn, lw["b_qkv"], y=pre.qkv), nqkv, h),
+        "o_gemm": (lambda: i4.int4_gemm(lw["w_o"], lw["s_o"], pre.attn, y=pre.y), h, h),
+        "gate_up_gemm": (lambda: i4.int4_gemm(lw["w_gu"], lw["s_gu"], pre.xn, y=pre.gu), 2 * inter, h),
+        "down_gemm": (lambda: i4.int4_gemm(lw["w_d"], lw["s_d"], pre.mlp, y=pre.y), h, inter),
+    }
+    peak_tf, peak_kind = measured_tensor_peak()
+    layer = {}
+    gemm_ms = 0.0
+    for name, (fn, N, K) in parts.items():
+        ms = timed(fn)
+        gemm_ms += ms
+        tf = 2.0 * n * N * K / (ms * 1e-3) / 1e12
+        layer[name] = {"us": round(ms * 1e3, 1), "TFLOPs": round(tf, 1), "frac_of_peak": round(tf / peak_tf, 4)}
+    layer["attention_causal"] = {"us": round(1e3 * timed(lambda: i4.paged_gqa_decode_strided(
+        pre.qkv, nqkv, shape.n_q, seq.k_pools[0], seq.v_pools[0], pre.tables, pre.ctx, pre.attn, pre.attn_ws)), 1)}
+    layer["glue"] = {"us": round(1e3 * timed(lambda: (
+        i4.rmsnorm(pre.y, lw["ln_post"], out=pre.xn, resid=pre.r), i4.silu_mul(pre.gu, out=pre.mlp),
+        i4.rope_kv_append(pre.qkv, pre.pos, shape.n_q, shape.n_kv, shape.theta))), 1)}
+    # the same prompt one token per step through the decode graph
+    seq2 = i4.Sequence(model, table, prompt)
+    graph = i4.DecodeGraph(model, seq2)
+    for _ in range(n):
         graph.replay()
     torch.cuda.synchronize()
-    seq.reset()
+    seq2.reset()
     e0.record()
-    for _ in range(len(prompt)):
+    for _ in range(n):
         graph.replay()
     e1.record()
     torch.cuda.synchronize()
     token_ms = e0.elapsed_time(e1)
-    first = int(seq.history[len(prompt)].item())
+    first = int(seq2.history[n].item())
     graph.close()
     err = i4.device_error()
-    print(json.dumps({"prefill": B, "prompt": len(prompt), "ttft_ms_chunked": round(chunked_ms, 2),
-                      "ttft_ms_token_by_token": round(token_ms, 2), "first_token_chunked": tok,
-                      "first_token_graph": first, "device_error": err}), flush=True)
+    layer_flops = 2.0 * n * (nqkv * h + h * h + 2 * inter * h + h * inter)
+    print(json.dumps({"prefill": "tcgen05", "prompt": n, "ttft_ms": round(ttft_ms, 2),
+                      "prompt_tok_s": round(n / (ttft_ms * 1e-3), 1),
+                      "gemm_flops_per_token_step": layer_flops * shape.layers,
+                      "gemm_TFLOPs_whole_prefill": round(layer_flops * shape.layers / (ttft_ms * 1e-3) / 1e12, 1),
+                      "tensor_peak_TFLOPs": peak_tf, "tensor_peak_kind": peak_kind,
+                      "layer0_parts": layer, "ttft_ms_token_by_token": round(token_ms, 2),
+                      "first_token_prefill": tok, "first_token_graph": first, "device_error": err}), flush=True)
     if tok != first or err:
         print(f"prefill: first tokens differ ({tok} vs {first}) or device error {err}", file=sys.stderr)
         return 1
     return 0
+
+
+def measured_tensor_peak():
+    """Dense fp16/bf16 tensor peak (TFLOP/s): the measured cuBLAS bf16 burst figure, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (cuBLAS bf16 burst; fp16 runs at the same rate)"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def main():
@@ -665,8 +717,8 @@ def main():
     ap.add_argument("--attention-sweep", action="store_true",
                     help="paged attention sweep over contexts, page sizes 16/64 and batches 1/8/32 (KV GB/s)")
     ap.add_argument("--sweep-contexts", default="512,2048,8192,32768")
-    ap.add_argument("--prefill", type=int, default=0,
-                    help="time to first token with this many prompt positions per step (e.g. 8)")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time to first token of a --prompt token prompt prefilled on the tcgen05 GEMM")
     ap.add_argument("--batched-decode", type=int, default=0,
                     help="decode this many sequences together (1..8) through the batched library calls")
     ap.add_argument("--gemv-batch", action="store_true",

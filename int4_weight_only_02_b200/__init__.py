@@ -294,4 +294,4 @@ def silu_mul(gate_up, out=None, stream=None):
     return out if gate_up.dim() == 2 else out.view(-1)
 
 
-from .runtime import BatchedDecode, DecodeGraph, DeviceModel, Sequence  # noqa: E402,F401
+from .runtime import BatchedDecode, DecodeGraph, DeviceModel, Prefill, Sequence  # noqa: E402,F401

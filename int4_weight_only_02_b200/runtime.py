@@ -193,7 +193,8 @@ class DecodeGraph:
 
 class BatchedDecode:
     """B sequences decoded together: one step is a CUDA graph of library calls -- embedding gather,
-    batched INT4 GEMVs (the B vectors as tensor-core columns where the shape allows), batched
+    batched INT4 linear layers (B <= 8: the B vectors as mma.sync columns where the shape allows; B > 8:
+    the tcgen05 GEMM), batched
     RMSNorm (+ residual), RoPE + K/V append, B-sequence paged attention reading q inside the qkv
     rows, SiLU-mul, lm_head and a per-row argmax that advances each sequence's position.
     Every sequence has its own page-table row over per-layer pools shared by the batch.
@@ -231,7 +232,7 @@ class BatchedDecode:
         # longer rows go through the register kernel, whose x stage holds a power-of-two number of vectors
         # at 68 bytes per 32 weights each, within 200 KB
         self.down_rows = B
-        if s.inter > 4096:
+        if s.inter > 4096 and B <= 8:  # more than 8 rows run on the tcgen05 GEMM, which takes any row length
             mr = 1
             while mr * 2 <= B and mr * 2 * (s.inter // 32) * 68 <= 200 * 1024:
                 mr *= 2
@@ -332,3 +333,93 @@ class BatchedDecode:
         self.tokens.copy_(torch.from_numpy(np.ascontiguousarray(tokens)))
         self.pos.copy_(torch.arange(c, c + self.B, dtype=torch.int32))
         self.ctx_len.copy_(torch.arange(c + 1, c + self.B + 1, dtype=torch.int32))
+
+
+class Prefill:
+    """Prompt prefill of one sequence with every prompt position at once.
+
+    Per layer the n prompt positions are n activation rows: batched RMSNorm, the qkv / o / gate-up / down
+    linear layers on the tcgen05 INT4 GEMM (``int4_gemm``), RoPE and the K/V append of all n positions into
+    the Sequence's own pages, causal paged attention (query row p over positions 0..p of the same pages, read
+    inside the qkv rows), SiLU-mul and the residual adds. The final norm and lm_head run for the last position
+    only; the argmax becomes the sequence's next token, so a DecodeGraph over the same Sequence continues at
+    position n. All launches go to one stream (no host synchronisation inside ``run``).
+    """
+
+    def __init__(self, model: DeviceModel, seq: Sequence, max_tokens: int = 512):
+        import torch
+        from . import paged_gqa_decode_ws_bytes
+        s, dev = model.shape, model.device
+        self.model, self.seq, self.shape = model, seq, s
+        self.n_max = n = int(max_tokens)
+        if n > s.max_ctx - 1:
+            raise ValueError(f"max_tokens {n} leaves no room for decoding within max_ctx {s.max_ctx}")
+        i32 = dict(dtype=torch.int32, device=dev)
+        f16 = dict(dtype=torch.float16, device=dev)
+        nqkv = (s.n_q + 2 * s.n_kv) * s.head_dim
+        self.tokens = torch.zeros(n, **i32)
+        self.pos = torch.arange(n, **i32)
+        self.ctx = torch.arange(1, n + 1, **i32)
+        # every row reads the sequence's own page-table row
+        self.tables = seq.page_table.view(1, -1).expand(n, -1).contiguous()
+        self.r = torch.zeros((n, s.hidden), **f16)
+        self.xn = torch.zeros((n, s.hidden), **f16)
+        self.qkv = torch.zeros((n, nqkv), **f16)
+        self.attn = torch.zeros((n, s.n_q * s.head_dim), **f16)
+        self.y = torch.zeros((n, s.hidden), **f16)
+        self.gu = torch.zeros((n, 2 * s.inter), **f16)
+        self.mlp = torch.zeros((n, s.inter), **f16)
+        self.logits = torch.zeros((1, s.vocab), dtype=torch.float32, device=dev)
+        # the attention workspace for any prompt length up to n (its split layout depends on the row count)
+        nbytes = max(paged_gqa_decode_ws_bytes(b, s.n_q, s.n_kv, s.head_dim, s.page_size, self.tables.shape[1])
+                     for b in range(1, n + 1))
+        self.attn_ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+
+    def run(self, prompt, stream=None):
+        """Enqueue the prefill of `prompt` (host ids or a device int32 tensor, 1 <= n <= max_tokens) on `stream`;
+        afterwards the Sequence holds the prompt's K/V, token = the first generated token, pos = n,
+        ctx_len = n + 1 and history[0..n] = prompt + that token."""
+        import torch
+        from . import (argmax_rows, embed_gather, int4_gemm, int4_gemv, paged_gqa_decode_strided, rmsnorm,
+                       rope_kv_append, silu_mul)
+        m, s, seq = self.model, self.shape, self.seq
+        g, L = m.glob, m.layers
+        if isinstance(prompt, torch.Tensor):
+            n = int(prompt.numel())
+            toks = prompt.to(device=m.device, dtype=torch.int32)
+        else:
+            prompt = np.asarray(prompt, dtype=np.int32)
+            n = len(prompt)
+            toks = torch.from_numpy(prompt).to(m.device)
+        if not 1 <= n <= self.n_max:
+            raise ValueError(f"prompt length {n} outside [1, {self.n_max}]")
+        nqkv = (s.n_q + 2 * s.n_kv) * s.head_dim
+        st = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(st):
+            self.tokens[:n].copy_(toks, non_blocking=True)
+            r, xn, qkv, attn, y, gu, mlp = (t[:n] for t in (self.r, self.xn, self.qkv, self.attn, self.y, self.gu,
+                                                            self.mlp))
+            embed_gather(g["embed"], self.tokens[:n], r, stream=st)
+            rmsnorm(r, L[0]["ln_in"], out=xn, eps=s.eps, stream=st)
+            for li, lw in enumerate(L):
+                int4_gemm(lw["w_qkv"], lw["s_qkv"], xn, lw["b_qkv"], y=qkv, stream=st)
+                rope_kv_append(qkv, self.pos[:n], s.n_q, s.n_kv, s.theta, seq.k_pools[li], seq.v_pools[li],
+                               self.tables[:n], stream=st)
+                paged_gqa_decode_strided(qkv, nqkv, s.n_q, seq.k_pools[li], seq.v_pools[li], self.tables[:n],
+                                         self.ctx[:n], attn, self.attn_ws, stream=st)
+                int4_gemm(lw["w_o"], lw["s_o"], attn, y=y, stream=st)
+                rmsnorm(y, lw["ln_post"], out=xn, resid=r, eps=s.eps, stream=st)
+                int4_gemm(lw["w_gu"], lw["s_gu"], xn, y=gu, stream=st)
+                silu_mul(gu, out=mlp, stream=st)
+                int4_gemm(lw["w_d"], lw["s_d"], mlp, y=y, stream=st)
+                gamma = L[li + 1]["ln_in"] if li + 1 < len(L) else g["ln_final"]
+                rmsnorm(y, gamma, out=xn, resid=r, eps=s.eps, stream=st)
+            # the last position's logits and the first generated token; the sequence continues at position n
+            int4_gemv(g["w_lm"], g["s_lm"], xn[n - 1:n], y=self.logits, out_fp32=True, stream=st)
+            seq.pos.fill_(n - 1)
+            seq.ctx_len.fill_(n)
+            argmax_rows(self.logits, seq.token, seq.pos, seq.ctx_len, stream=st)
+            seq.history[:n].copy_(self.tokens[:n], non_blocking=True)
+            seq.history[n:n + 1].copy_(seq.token, non_blocking=True)
+            seq.status.zero_()
+        return seq.token
