@@ -632,11 +632,12 @@ def run_prefill(args):
 
     lw = model.layers[0]
     h, inter, nqkv = shape.hidden, shape.inter, shape.qkv_rows
+    ws = pre.gemm_ws  # the split-K workspace the prefill itself uses
     parts = {
-        "qkv_gemm": (lambda: i4.int4_gemm(lw["w_qkv"], lw["s_qkv"], pre.xn, lw["b_qkv"], y=pre.qkv), nqkv, h),
-        "o_gemm": (lambda: i4.int4_gemm(lw["w_o"], lw["s_o"], pre.attn, y=pre.y), h, h),
-        "gate_up_gemm": (lambda: i4.int4_gemm(lw["w_gu"], lw["s_gu"], pre.xn, y=pre.gu), 2 * inter, h),
-        "down_gemm": (lambda: i4.int4_gemm(lw["w_d"], lw["s_d"], pre.mlp, y=pre.y), h, inter),
+        "qkv_gemm": (lambda: i4.int4_gemm(lw["w_qkv"], lw["s_qkv"], pre.xn, lw["b_qkv"], y=pre.qkv, ws=ws), nqkv, h),
+        "o_gemm": (lambda: i4.int4_gemm(lw["w_o"], lw["s_o"], pre.attn, y=pre.y, ws=ws), h, h),
+        "gate_up_gemm": (lambda: i4.int4_gemm(lw["w_gu"], lw["s_gu"], pre.xn, y=pre.gu, ws=ws), 2 * inter, h),
+        "down_gemm": (lambda: i4.int4_gemm(lw["w_d"], lw["s_d"], pre.mlp, y=pre.y, ws=ws), h, inter),
     }
     peak_tf, peak_kind = measured_tensor_peak()
     layer = {}

@@ -82,11 +82,21 @@ I4_API int int4_gemv(const uint32_t *w, const uint16_t *scales, const uint16_t *
  * memory; y = accumulator (+ bias), stored as fp16 or fp32.
  *   w [N][K/8] uint32 and x [M][K] fp16, 16-byte aligned; scales [N][K/128];
  *   bias [N] or NULL; y [M][N]. group == 128, K % 128 == 0, K <= 65536.
+ * The weights enter the product exactly: each dequantised weight q * s is
+ * held as two fp16 terms, hi = fp16(q * s) and lo = q * s - hi (exact), both
+ * multiplied into the same fp32 accumulator.
  * Any M >= 1 (tiles of 16 .. 512 activation rows per CTA); the tensor maps of
  * w and x are encoded on the host at each call.
+ *   ws, ws_bytes: optional workspace (256-byte aligned) of
+ *   int4_gemm_ws_bytes(M, N, K) bytes (0 when the shape is not split). With
+ *   it, shapes whose 128-row tiles leave SMs idle split K over several CTAs,
+ *   and a second kernel adds their fp32 partials in split order; without it
+ *   (NULL) K is not split. Calls sharing one workspace must not overlap on
+ *   the GPU.
  */
+I4_API size_t int4_gemm_ws_bytes(int M, int N, int K);
 I4_API int int4_gemm(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
-                     int y_is_fp32, int M, int N, int K, int group, void *stream);
+                     int y_is_fp32, int M, int N, int K, int group, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Test export: q[n][k] = signed field of w (bit-exact unpack check).

@@ -64,7 +64,8 @@ _SIGS = {
     "i4_last_error": (ctypes.c_char_p, []),
     "i4_version": (ctypes.c_char_p, []),
     "int4_gemv": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
-    "int4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "int4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "int4_gemm_ws_bytes": (_sz, [_i, _i, _i]),
     "i4_int4_gemv_variant": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "i4_int4_unpack": (_i, [_vp, _vp, _i, _i, _vp]),
     "paged_gqa_decode_ws_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
@@ -163,14 +164,20 @@ def int4_gemv(w, scales, x, bias=None, y=None, out_fp32: bool = False, group: in
     return y if x.dim() == 2 else y.view(-1)
 
 
-def int4_gemm(w, scales, x, bias=None, y=None, out_fp32: bool = False, group: int = 128, stream=None):
-    """y[M][N] = x[M][K] . dequant(w, scales)^T (+ bias) on the tcgen05 tensor cores (any M)."""
+def int4_gemm_ws_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().int4_gemm_ws_bytes(M, N, K))
+
+
+def int4_gemm(w, scales, x, bias=None, y=None, out_fp32: bool = False, group: int = 128, ws=None, stream=None):
+    """y[M][N] = x[M][K] . dequant(w, scales)^T (+ bias) on the tcgen05 tensor cores (any M). With `ws` (a
+    zeroed uint8 device tensor of at least int4_gemm_ws_bytes(M, N, K) bytes) K may be split over CTAs."""
     import torch
     M, K = x.shape
     N = w.shape[0]
     if y is None:
         y = torch.empty((M, N), device=x.device, dtype=torch.float32 if out_fp32 else torch.float16)
-    _check(lib().int4_gemm(_p(w), _p(scales), _p(x), _p(bias), _p(y), int(out_fp32), M, N, K, group,
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().int4_gemm(_p(w), _p(scales), _p(x), _p(bias), _p(y), int(out_fp32), M, N, K, group, _p(ws), nb,
                            _stream(stream)), "int4_gemm")
     return y
 

@@ -13,15 +13,22 @@
 //   warp 0     one thread issues TMA copies per 64-wide K chunk: the raw INT4
 //              rows (128 x 32 bytes) and the fp16 activation rows (BN x 128
 //              bytes, 128-byte swizzle), completing on an mbarrier;
-//   warps 2-5  thread t dequantises weight row t of the chunk: fp16(q * s),
-//              written in the same 128-byte-swizzled K-major layout;
+//   warps 2-9  threads t and t + 128 dequantise the two halves of weight row t
+//              of the chunk into two fp16 tiles in the same 128-byte-swizzled
+//              K-major layout:
+//              hi = fp16(q * s) and lo = fma(q, s, -hi), the exact remainder
+//              (q * s has at most 14 significant bits), so hi + lo = q * s;
 //   warp 1     allocates the TMEM columns, and one thread issues
 //              tcgen05.mma (kind::f16, M = 128, N = min(BN, 256), K = 16) on
-//              shared-memory descriptors, committing each stage back to an
-//              mbarrier so its buffers can be refilled;
+//              shared-memory descriptors for both tiles into one accumulator,
+//              committing each stage back to an mbarrier so its buffers can be
+//              refilled;
 //   warps 2-5  finally read their 32 TMEM lanes each (tcgen05.ld) and store y.
-// Dequantised weights are rounded to fp16 once (q * s) before the product; the
-// accumulation is fp32. No multicast; one GPU.
+// Every product q * s * x is exact in the fp32 accumulation. When the tiles of
+// a layer are too few to fill the GPU, K is split over gridDim.z CTAs: each
+// writes its fp32 partial of y to the caller's workspace and a second, fully
+// parallel kernel adds the partials in split order with the bias and stores y.
+// No multicast; one GPU.
 #include <cuda.h>
 
 #include <mutex>
@@ -35,9 +42,10 @@ namespace i4 {
 
 constexpr int kGBM = 128;           // weight rows per CTA (MMA M)
 constexpr int kGBK = 64;            // K per stage: one 128-byte row of fp16
-constexpr int kGThreads = 192;
+constexpr int kGDeqWarps = 8;       // dequantisation warps: two per weight row, four words each
+constexpr int kGThreads = 64 + 32 * kGDeqWarps;
 constexpr int kGMaxStages = 6;
-constexpr unsigned kGATile = kGBM * kGBK * 2;  // dequantised weights, 16 KB
+constexpr unsigned kGATile = kGBM * kGBK * 2;  // one dequantised weight tile (hi or lo), 16 KB
 constexpr unsigned kGRaw = kGBM * kGBK / 2;    // raw INT4 rows, 4 KB
 
 __device__ int g_gemm_error = 0;
@@ -109,12 +117,14 @@ struct GemmArgs {
     const uint16_t *scales, *bias;
     void *y;
     int y_fp32, M, N, K, stages;
+    int chunks_per_split;  // K chunks of one split (gridDim.z splits)
+    float *part;           // split partials [split][M][N] fp32 (splits > 1)
 };
 
-// Dynamic shared memory per stage (1024-byte aligned): A tile 16 KB | B tile BN x 128 B | raw INT4 4 KB.
+// Dynamic shared memory per stage (1024-byte aligned): A hi 16 KB | A lo 16 KB | B tile BN x 128 B | raw INT4 4 KB.
 template <int BN>
 __host__ __device__ constexpr unsigned gemm_stage_bytes() {
-    return kGATile + (unsigned)BN * 128u + kGRaw;
+    return 2 * kGATile + (unsigned)BN * 128u + kGRaw;
 }
 
 template <int BN>
@@ -129,19 +139,23 @@ __global__ void __launch_bounds__(kGThreads, 1)
     __shared__ __align__(8) uint64_t raw_full[kGMaxStages], a_full[kGMaxStages], empty[kGMaxStages], acc_full;
     __shared__ uint32_t tmem_base;
 
-    const int S = a.stages, K = a.K, n_chunks = K / kGBK;
+    const int S = a.stages, K = a.K;
+    const int c_begin = blockIdx.z * a.chunks_per_split;
+    const int c_end = (c_begin + a.chunks_per_split) < K / kGBK ? (c_begin + a.chunks_per_split) : K / kGBK;
+    const int n_chunks = c_end > c_begin ? c_end - c_begin : 0;
     const int n0 = blockIdx.x * kGBM, m0 = blockIdx.y * BN;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     auto stage_a = [&](int s) { return smem + (size_t)s * gemm_stage_bytes<BN>(); };
-    auto stage_b = [&](int s) { return stage_a(s) + kGATile; };
+    auto stage_lo = [&](int s) { return stage_a(s) + kGATile; };
+    auto stage_b = [&](int s) { return stage_a(s) + 2 * kGATile; };
     auto stage_raw = [&](int s) { return stage_b(s) + (size_t)BN * 128; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&raw_full[s], 1);
-            mbar_init(&a_full[s], 4);
+            mbar_init(&a_full[s], kGDeqWarps);
             mbar_init(&empty[s], 1);
         }
         mbar_init(&acc_full, 1);
@@ -168,11 +182,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     break;
                 }
                 if (gemm_aborted()) break;
+                const int kc = c_begin + c;
                 mbar_expect_tx(&raw_full[s], kGRaw + (unsigned)BN * 128u);
-                tma_load_2d(stage_raw(s), &tm_w, c * (kGBK / 2), n0, &raw_full[s]);
+                tma_load_2d(stage_raw(s), &tm_w, kc * (kGBK / 2), n0, &raw_full[s]);
 #pragma unroll
                 for (int h = 0; h < BN / (int)XBOX; ++h)
-                    tma_load_2d(stage_b(s) + (size_t)h * XBOX * 128, &tm_x, c * kGBK, m0 + h * (int)XBOX, &raw_full[s]);
+                    tma_load_2d(stage_b(s) + (size_t)h * XBOX * 128, &tm_x, kc * kGBK, m0 + h * (int)XBOX, &raw_full[s]);
             }
         }
     } else if (warp == 1) {
@@ -186,85 +201,113 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     break;
                 }
                 fence_after_sync();
-                const uint32_t sa = smem_u32(stage_a(s)), sb = smem_u32(stage_b(s));
+                const uint32_t sa = smem_u32(stage_a(s)), sl = smem_u32(stage_lo(s)), sb = smem_u32(stage_b(s));
 #pragma unroll
                 for (int kk = 0; kk < kGBK / 16; ++kk) {
-                    const uint64_t ad = desc_sw128(sa + 32 * kk);
+                    const uint64_t ad = desc_sw128(sa + 32 * kk), ld = desc_sw128(sl + 32 * kk);
 #pragma unroll
-                    for (int h = 0; h < NHALF; ++h)
-                        umma_f16(tmem + (uint32_t)(h * NMMA), ad, desc_sw128(sb + (uint32_t)(h * NMMA * 128) + 32 * kk),
-                                 idesc, (c > 0 || kk > 0) ? 1 : 0);
+                    for (int h = 0; h < NHALF; ++h) {
+                        const uint64_t bd = desc_sw128(sb + (uint32_t)(h * NMMA * 128) + 32 * kk);
+                        umma_f16(tmem + (uint32_t)(h * NMMA), ad, bd, idesc, (c > 0 || kk > 0) ? 1 : 0);
+                        umma_f16(tmem + (uint32_t)(h * NMMA), ld, bd, idesc, 1);
+                    }
                 }
                 umma_commit(&empty[s]);  // the stage's buffers are free once these MMAs have read them
             }
             umma_commit(&acc_full);  // every MMA issued above has completed
         }
     } else {
-        // ---------------- dequantisation (thread t: weight row t of the tile), then the epilogue
-        const int t = threadIdx.x - 64;
+        // ---------------- dequantisation (threads t, t + 128: the two halves of weight row t), then the
+        // epilogue (warps 2-5)
+        const int td = threadIdx.x - 64, t = td & 127, half = td >> 7;
         const int n = n0 + t, groups = K >> 7;
         const bool row_ok = n < a.N;
         const uint16_t *srow = a.scales + (size_t)(row_ok ? n : 0) * groups;
-        uint16_t s_next = row_ok ? ldg_u16(srow) : 0;
+        uint16_t s_next = (row_ok && n_chunks > 0) ? ldg_u16(srow + (c_begin * kGBK >> 7)) : 0;
         bool ok = true;
         for (int c = 0; c < n_chunks; ++c) {
             const int s = c % S, use = c / S;
             const uint16_t sc = s_next;
-            if (c + 1 < n_chunks) s_next = row_ok ? ldg_u16(srow + ((c + 1) * kGBK >> 7)) : 0;
+            if (c + 1 < n_chunks) s_next = row_ok ? ldg_u16(srow + ((c_begin + c + 1) * kGBK >> 7)) : 0;
             if (ok && !mbar_wait(&raw_full[s], (unsigned)(use & 1))) {
                 record_error(&g_gemm_error, 1);
                 ok = false;
             }
             if (ok) {
-                const uint4 *raw = reinterpret_cast<const uint4 *>(stage_raw(s) + (size_t)t * 32);
-                const uint4 r0 = raw[0], r1 = raw[1];
-                const uint32_t words[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+                const uint4 r0 = *reinterpret_cast<const uint4 *>(stage_raw(s) + (size_t)t * 32 + 16 * half);
+                const uint32_t words[4] = {r0.x, r0.y, r0.z, r0.w};
                 const uint32_t s2 = (uint32_t)sc | ((uint32_t)sc << 16);
-                unsigned char *arow = stage_a(s) + (size_t)(t >> 3) * 1024 + (size_t)(t & 7) * 128;
+                const size_t roff = (size_t)(t >> 3) * 1024 + (size_t)(t & 7) * 128;
+                unsigned char *arow = stage_a(s) + roff, *lrow = stage_lo(s) + roff;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {  // word j: k = 8j .. 8j + 7 of the chunk -> 16-byte chunk j
+                for (int jj = 0; jj < 4; ++jj) {  // word j: k = 8j .. 8j + 7 of the chunk -> 16-byte chunk j
+                    const int j = 4 * half + jj;
                     uint32_t q[4];
-                    unpack_word_exact(words[j], q);  // (k0,k4) (k1,k5) (k2,k6) (k3,k7), exact integers
-                    uint32_t w[4];
+                    unpack_word_exact(words[jj], q);  // (k0,k4) (k1,k5) (k2,k6) (k3,k7), exact integers
+                    uint32_t w[4], r[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const __half2 p = __hmul2(*reinterpret_cast<const __half2 *>(&q[e]),
-                                                  *reinterpret_cast<const __half2 *>(&s2));
-                        w[e] = *reinterpret_cast<const uint32_t *>(&p);
+                        const __half2 qh = *reinterpret_cast<const __half2 *>(&q[e]);
+                        const __half2 sh = *reinterpret_cast<const __half2 *>(&s2);
+                        const __half2 hi = __hmul2(qh, sh);
+                        const __half2 lo = __hfma2(qh, sh, __hneg2(hi));  // q * s - hi, exact
+                        w[e] = *reinterpret_cast<const uint32_t *>(&hi);
+                        r[e] = *reinterpret_cast<const uint32_t *>(&lo);
                     }
-                    const uint4 nat = make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
-                                                 __byte_perm(w[0], w[1], 0x7632), __byte_perm(w[2], w[3], 0x7632));
-                    *reinterpret_cast<uint4 *>(arow + ((j ^ (t & 7)) << 4)) = nat;
+                    const int pos16 = (j ^ (t & 7)) << 4;
+                    *reinterpret_cast<uint4 *>(arow + pos16) =
+                        make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
+                                   __byte_perm(w[0], w[1], 0x7632), __byte_perm(w[2], w[3], 0x7632));
+                    *reinterpret_cast<uint4 *>(lrow + pos16) =
+                        make_uint4(__byte_perm(r[0], r[1], 0x5410), __byte_perm(r[2], r[3], 0x5410),
+                                   __byte_perm(r[0], r[1], 0x7632), __byte_perm(r[2], r[3], 0x7632));
                 }
             }
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[s]);
         }
-        // epilogue: TMEM lane 32 * (warp % 4) + lane holds row n0 + that lane, columns = tokens m0 ..
+        // epilogue (warps 2-5): TMEM lane 32 * (warp % 4) + lane holds row n0 + that lane, columns = tokens m0 ..
+        if (warp < 6) {
         if (!mbar_wait(&acc_full, 0u)) record_error(&g_gemm_error, 1);
         fence_after_sync();
-        if (!gemm_aborted()) {
-            const int row = 32 * (warp & 3) + lane, nn = n0 + row;
-            const float bias = (a.bias && nn < a.N) ? half_bits_to_float(a.bias[nn]) : 0.f;
-            const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const int row = 32 * (warp & 3) + lane, nn = n0 + row;
+        const float bias = (a.bias && nn < a.N) ? half_bits_to_float(a.bias[nn]) : 0.f;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        auto store = [&](int m, float v) {
+            if (a.y_fp32)
+                reinterpret_cast<float *>(a.y)[(size_t)m * a.N + nn] = v + bias;
+            else
+                reinterpret_cast<uint16_t *>(a.y)[(size_t)m * a.N + nn] = float_to_half_bits(v + bias);
+        };
+        if (gridDim.z == 1) {
+            if (!__any_sync(0xffffffffu, gemm_aborted())) {  // warp-uniform around the warp-wide tcgen05.ld
 #pragma unroll 1
-            for (int j0 = 0; j0 < BN; j0 += 16) {
-                float v[16];
-                tmem_ld16(taddr + (uint32_t)j0, v);
-                if (nn < a.N) {
+                for (int j0 = 0; j0 < BN; j0 += 16) {
+                    float v[16];
+                    tmem_ld16(taddr + (uint32_t)j0, v);
+                    if (nn < a.N) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int m = m0 + j0 + i;
-                        if (m < a.M) {
-                            if (a.y_fp32)
-                                reinterpret_cast<float *>(a.y)[(size_t)m * a.N + nn] = v[i] + bias;
-                            else
-                                reinterpret_cast<uint16_t *>(a.y)[(size_t)m * a.N + nn] = float_to_half_bits(v[i] + bias);
-                        }
+                        for (int i = 0; i < 16; ++i)
+                            if (m0 + j0 + i < a.M) store(m0 + j0 + i, v[i]);
                     }
                 }
             }
+        } else {
+            // split K: this split's partial tile to the workspace, [split][m][n] fp32 (coalesced over the
+            // rows n); gemm_reduce_kernel sums the splits in order afterwards
+            float *mine = a.part + (size_t)blockIdx.z * a.M * a.N;
+#pragma unroll 1
+            for (int j0 = 0; j0 < BN; j0 += 16) {
+                float v[16];
+                tmem_ld16(taddr + (uint32_t)j0, v);  // warp-wide: every lane takes part
+                if (nn < a.N) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (m0 + j0 + i < a.M) mine[(size_t)(m0 + j0 + i) * a.N + nn] = v[i];
+                }
+            }
+        }
         }
     }
     fence_before_sync();
@@ -272,6 +315,39 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (warp == 1) {
         fence_after_sync();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS) : "memory");
+    }
+}
+
+// y[m][n] = sum_z part[z][m][n] (+ bias[n]), the splits added in order; 8 outputs per thread.
+__global__ void gemm_reduce_kernel(const float *part, const uint16_t *bias, void *y, int y_fp32, int M, int N,
+                                   int splits) {
+    const size_t total = (size_t)M * N;
+    for (size_t i = (size_t)(blockIdx.x * blockDim.x + threadIdx.x) * 8; i < total;
+         i += (size_t)gridDim.x * blockDim.x * 8) {
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        const int n0 = (int)(i % N);
+        for (int z = 0; z < splits; ++z) {
+            const float *pz = part + (size_t)z * total + i;
+            if (i + 8 <= total && ((reinterpret_cast<uintptr_t>(pz) & 15) == 0)) {
+                const float4 u = __ldcs(reinterpret_cast<const float4 *>(pz));
+                const float4 w = __ldcs(reinterpret_cast<const float4 *>(pz + 4));
+                acc[0] += u.x; acc[1] += u.y; acc[2] += u.z; acc[3] += u.w;
+                acc[4] += w.x; acc[5] += w.y; acc[6] += w.z; acc[7] += w.w;
+            } else {
+                for (int e = 0; e < 8 && i + e < total; ++e) acc[e] += __ldcs(pz + e);
+            }
+        }
+        for (int e = 0; e < 8 && i + e < total; ++e) {
+            int n = n0 + e;
+            if (n >= N) n -= N;
+            const float v = acc[e] + (bias ? half_bits_to_float(bias[n]) : 0.f);
+            if (y_fp32)
+                reinterpret_cast<float *>(y)[i + e] = v;
+            else
+                reinterpret_cast<uint16_t *>(y)[i + e] = float_to_half_bits(v);
+        }
     }
 }
 
@@ -311,9 +387,40 @@ static int make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, in
     return I4_OK;
 }
 
+// Splits of K for a grid of `tiles` output tiles: enough CTAs to cover the SMs, each split at least 8 chunks.
+static int gemm_splits(int tiles, int chunks, int sms) {
+    int ks = (sms + tiles - 1) / tiles;
+    const int cap = chunks / 8 > 1 ? chunks / 8 : 1;
+    ks = ks < cap ? ks : cap;
+    return ks < 1 ? 1 : ks;
+}
+
+static int gemm_bn(int M) {
+    return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : M <= 256 ? 256 : 512;
+}
+
+static int num_sms() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms < 1) sms = kNumSMs;
+    }
+    return sms;
+}
+
+size_t gemm_ws_bytes(int M, int N, int K) {
+    const int BN = gemm_bn(M);
+    const int tiles = ((N + kGBM - 1) / kGBM) * ((M + BN - 1) / BN);
+    const int ks = gemm_splits(tiles, K / kGBK, num_sms());
+    if (ks == 1) return 0;
+    return (size_t)ks * M * N * sizeof(float);
+}
+
 template <int BN>
 static int launch_gemm_bn(const uint32_t *w, const uint16_t *s, const uint16_t *x, const uint16_t *bias, void *y,
-                          int y_fp32, int M, int N, int K, cudaStream_t stream) {
+                          int y_fp32, int M, int N, int K, void *ws, size_t ws_bytes, cudaStream_t stream) {
     CUtensorMap tw, tx;
     int st = make_map(&tw, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K / 2, (uint64_t)N, kGBK / 2, kGBM,
                       CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -338,20 +445,39 @@ static int launch_gemm_bn(const uint32_t *w, const uint16_t *s, const uint16_t *
         if (e != cudaSuccess) return cuda_check(e, "int4_gemm smem attribute");
         configured = (int)smem;
     }
-    GemmArgs a = {s, bias, y, y_fp32, M, N, K, stages};
-    const dim3 grid((N + kGBM - 1) / kGBM, (M + BN - 1) / BN);
+    const int tiles_n = (N + kGBM - 1) / kGBM, tiles_m = (M + BN - 1) / BN;
+    int ks = 1;
+    GemmArgs a = {s, bias, y, y_fp32, M, N, K, stages, chunks, nullptr};
+    if (ws) {  // split K over the caller's workspace when the tiles alone leave SMs idle
+        ks = gemm_splits(tiles_n * tiles_m, chunks, num_sms());
+        if (ks > 1) {
+            const size_t need = gemm_ws_bytes(M, N, K);
+            if (ws_bytes < need) return fail(I4_EINVAL, "int4_gemm: workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+            a.part = reinterpret_cast<float *>(ws);
+            a.chunks_per_split = (chunks + ks - 1) / ks;
+            ks = (chunks + a.chunks_per_split - 1) / a.chunks_per_split;
+        }
+    }
+    const dim3 grid(tiles_n, tiles_m, ks);
     i4_gemm_tc_kernel<BN><<<grid, kGThreads, smem, stream>>>(tw, tx, a);
-    return launch_check("int4_gemm");
+    int st2 = launch_check("int4_gemm");
+    if (st2 || ks == 1) return st2;
+    const size_t outs = (size_t)M * N;
+    const int blocks = (int)((outs / 8 + 255) / 256) < 4 * num_sms() ? (int)((outs / 8 + 255) / 256) : 4 * num_sms();
+    gemm_reduce_kernel<<<blocks > 0 ? blocks : 1, 256, 0, stream>>>(a.part, bias, y, y_fp32, M, N, ks);
+    return launch_check("int4_gemm split-K reduction");
 }
 
 int launch_int4_gemm(const uint32_t *w, const uint16_t *s, const uint16_t *x, const uint16_t *bias, void *y,
-                     int y_fp32, int M, int N, int K, cudaStream_t stream) {
-    if (M <= 16) return launch_gemm_bn<16>(w, s, x, bias, y, y_fp32, M, N, K, stream);
-    if (M <= 32) return launch_gemm_bn<32>(w, s, x, bias, y, y_fp32, M, N, K, stream);
-    if (M <= 64) return launch_gemm_bn<64>(w, s, x, bias, y, y_fp32, M, N, K, stream);
-    if (M <= 128) return launch_gemm_bn<128>(w, s, x, bias, y, y_fp32, M, N, K, stream);
-    if (M <= 256) return launch_gemm_bn<256>(w, s, x, bias, y, y_fp32, M, N, K, stream);
-    return launch_gemm_bn<512>(w, s, x, bias, y, y_fp32, M, N, K, stream);
+                     int y_fp32, int M, int N, int K, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    switch (gemm_bn(M)) {
+        case 16: return launch_gemm_bn<16>(w, s, x, bias, y, y_fp32, M, N, K, ws, ws_bytes, stream);
+        case 32: return launch_gemm_bn<32>(w, s, x, bias, y, y_fp32, M, N, K, ws, ws_bytes, stream);
+        case 64: return launch_gemm_bn<64>(w, s, x, bias, y, y_fp32, M, N, K, ws, ws_bytes, stream);
+        case 128: return launch_gemm_bn<128>(w, s, x, bias, y, y_fp32, M, N, K, ws, ws_bytes, stream);
+        case 256: return launch_gemm_bn<256>(w, s, x, bias, y, y_fp32, M, N, K, ws, ws_bytes, stream);
+        default: return launch_gemm_bn<512>(w, s, x, bias, y, y_fp32, M, N, K, ws, ws_bytes, stream);
+    }
 }
 
 int read_gemm_error(int reset) {
@@ -370,8 +496,13 @@ int read_gemm_error(int reset) {
 
 using namespace i4;
 
+extern "C" size_t int4_gemm_ws_bytes(int M, int N, int K) {
+    if (M < 1 || N < 1 || K < 128 || K % 128) return 0;
+    return gemm_ws_bytes(M, N, K);
+}
+
 extern "C" int int4_gemm(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
-                         int y_is_fp32, int M, int N, int K, int group, void *stream) {
+                         int y_is_fp32, int M, int N, int K, int group, void *ws, size_t ws_bytes, void *stream) {
     if (!w || !scales || !x || !y) return fail(I4_EINVAL, "int4_gemm: null pointer");
     if (M < 1 || N < 1 || K < 1) return fail(I4_EINVAL, "int4_gemm: M, N, K must be positive");
     if (group != 128) return fail(I4_EUNSUPPORTED, "int4_gemm: group %d (only 128)", group);
@@ -379,6 +510,7 @@ extern "C" int int4_gemm(const uint32_t *w, const uint16_t *scales, const uint16
     if (K > 65536 || N > (1 << 24) || M > (1 << 20)) return fail(I4_EUNSUPPORTED, "int4_gemm: shape too large");
     if (!aligned(w, 16) || !aligned(x, 16) || !aligned(scales, 2) || !aligned(y, y_is_fp32 ? 4 : 2))
         return fail(I4_EALIGN, "int4_gemm: w and x must be 16-byte aligned");
+    if (ws && !aligned(ws, 256)) return fail(I4_EALIGN, "int4_gemm: workspace must be 256-byte aligned");
     if (g_dry_run) return I4_OK;
-    return launch_int4_gemm(w, scales, x, bias, y, y_is_fp32, M, N, K, (cudaStream_t)stream);
+    return launch_int4_gemm(w, scales, x, bias, y, y_is_fp32, M, N, K, ws, ws_bytes, (cudaStream_t)stream);
 }

@@ -225,12 +225,12 @@ static int gemv_entry(const uint32_t *w, const uint16_t *scales, const uint16_t 
 }
 
 extern "C" int int4_gemm(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
-                         int y_is_fp32, int M, int N, int K, int group, void *stream);
+                         int y_is_fp32, int M, int N, int K, int group, void *ws, size_t ws_bytes, void *stream);
 
 extern "C" int int4_gemv(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias, void *y,
                          int y_is_fp32, int M, int N, int K, int group, void *stream) {
     // more than 8 activation rows: a dense contraction, on the tcgen05 GEMM
-    if (M > 8) return int4_gemm(w, scales, x, bias, y, y_is_fp32, M, N, K, group, stream);
+    if (M > 8) return int4_gemm(w, scales, x, bias, y, y_is_fp32, M, N, K, group, nullptr, 0, stream);
     return gemv_entry(w, scales, x, bias, y, y_is_fp32, M, N, K, group, -1, 0, (cudaStream_t)stream);
 }
 

@@ -26,6 +26,17 @@ def to_device(a: np.ndarray, device="cuda"):
     return torch.from_numpy(np.ascontiguousarray(a)).to(device)
 
 
+def _gemm_workspace(s, rows: int, dev):
+    """A zeroed split-K workspace for every linear layer of the model at `rows` activation rows."""
+    import torch
+    from . import int4_gemm_ws_bytes
+    nqkv = (s.n_q + 2 * s.n_kv) * s.head_dim
+    shapes = [(nqkv, s.hidden), (s.hidden, s.n_q * s.head_dim), (2 * s.inter, s.hidden), (s.hidden, s.inter),
+              (s.vocab, s.hidden)]
+    nbytes = max(int4_gemm_ws_bytes(rows, n, k) for n, k in shapes)
+    return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+
+
 class DeviceModel:
     def __init__(self, shape: synth.ModelShape, layers, glob, device="cuda"):
         self.shape = shape
@@ -227,6 +238,7 @@ class BatchedDecode:
         self.logits = torch.zeros((B, s.vocab), dtype=torch.float32, device=dev)
         nbytes = paged_gqa_decode_ws_bytes(B, s.n_q, s.n_kv, s.head_dim, s.page_size, page_tables.shape[1])
         self.attn_ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        self.gemm_ws = _gemm_workspace(s, B, dev) if B > 8 else None
         self.graph = None
         # vectors per down-projection call: the batched tensor-core GEMV takes rows of up to 4096 weights;
         # longer rows go through the register kernel, whose x stage holds a power-of-two number of vectors
@@ -245,10 +257,16 @@ class BatchedDecode:
         self.pos.zero_()
         self.ctx_len.fill_(1)
 
+    def _linear(self, w, sc, x, bias=None, y=None, out_fp32=False, stream=None):
+        from . import int4_gemm, int4_gemv
+        if self.B > 8:  # the tcgen05 GEMM, K split over CTAs where the tiles leave SMs idle
+            return int4_gemm(w, sc, x, bias, y=y, out_fp32=out_fp32, ws=self.gemm_ws, stream=stream)
+        return int4_gemv(w, sc, x, bias, y=y, out_fp32=out_fp32, stream=stream)
+
     def step(self, stream=None):
         """Enqueue one decode step of all B sequences on `stream` (no allocation, capturable)."""
-        from . import (argmax_rows, embed_gather, int4_gemv, paged_gqa_decode_strided, rmsnorm,
-                       rope_kv_append, silu_mul)
+        from . import argmax_rows, embed_gather, paged_gqa_decode_strided, rmsnorm, rope_kv_append, silu_mul
+        int4_gemv = self._linear
         m, s = self.model, self.shape
         g, L = m.glob, m.layers
         nqkv = (s.n_q + 2 * s.n_kv) * s.head_dim
@@ -374,6 +392,7 @@ class Prefill:
         nbytes = max(paged_gqa_decode_ws_bytes(b, s.n_q, s.n_kv, s.head_dim, s.page_size, self.tables.shape[1])
                      for b in range(1, n + 1))
         self.attn_ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        self.gemm_ws = _gemm_workspace(s, n, dev)
 
     def run(self, prompt, stream=None):
         """Enqueue the prefill of `prompt` (host ids or a device int32 tensor, 1 <= n <= max_tokens) on `stream`;
@@ -402,16 +421,16 @@ class Prefill:
             embed_gather(g["embed"], self.tokens[:n], r, stream=st)
             rmsnorm(r, L[0]["ln_in"], out=xn, eps=s.eps, stream=st)
             for li, lw in enumerate(L):
-                int4_gemm(lw["w_qkv"], lw["s_qkv"], xn, lw["b_qkv"], y=qkv, stream=st)
+                int4_gemm(lw["w_qkv"], lw["s_qkv"], xn, lw["b_qkv"], y=qkv, ws=self.gemm_ws, stream=st)
                 rope_kv_append(qkv, self.pos[:n], s.n_q, s.n_kv, s.theta, seq.k_pools[li], seq.v_pools[li],
                                self.tables[:n], stream=st)
                 paged_gqa_decode_strided(qkv, nqkv, s.n_q, seq.k_pools[li], seq.v_pools[li], self.tables[:n],
                                          self.ctx[:n], attn, self.attn_ws, stream=st)
-                int4_gemm(lw["w_o"], lw["s_o"], attn, y=y, stream=st)
+                int4_gemm(lw["w_o"], lw["s_o"], attn, y=y, ws=self.gemm_ws, stream=st)
                 rmsnorm(y, lw["ln_post"], out=xn, resid=r, eps=s.eps, stream=st)
-                int4_gemm(lw["w_gu"], lw["s_gu"], xn, y=gu, stream=st)
+                int4_gemm(lw["w_gu"], lw["s_gu"], xn, y=gu, ws=self.gemm_ws, stream=st)
                 silu_mul(gu, out=mlp, stream=st)
-                int4_gemm(lw["w_d"], lw["s_d"], mlp, y=y, stream=st)
+                int4_gemm(lw["w_d"], lw["s_d"], mlp, y=y, ws=self.gemm_ws, stream=st)
                 gamma = L[li + 1]["ln_in"] if li + 1 < len(L) else g["ln_final"]
                 rmsnorm(y, gamma, out=xn, resid=r, eps=s.eps, stream=st)
             # the last position's logits and the first generated token; the sequence continues at position n

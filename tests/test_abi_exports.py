@@ -45,10 +45,12 @@ def test_host_validation_without_gpu(i4lib):
     assert L.int4_gemv(fake, fake, fake, None, fake, 0, 1, 16, 100, 128, None) == i4lib.I4_EINVAL
     # more than 8 rows go to the tcgen05 GEMM, which validates the same way before any launch
     assert L.int4_gemv(fake, fake, fake, None, fake, 0, 9, 16, 128, 64, None) == i4lib.I4_EUNSUPPORTED
-    assert L.int4_gemm(fake, fake, fake, None, fake, 0, 512, 16, 100, 128, None) == i4lib.I4_EINVAL
-    assert L.int4_gemm(ctypes.c_void_p((1 << 20) + 8), fake, fake, None, fake, 0, 512, 16, 128, 128,
+    assert L.int4_gemm(fake, fake, fake, None, fake, 0, 512, 16, 100, 128, None, 0, None) == i4lib.I4_EINVAL
+    assert L.int4_gemm(ctypes.c_void_p((1 << 20) + 8), fake, fake, None, fake, 0, 512, 16, 128, 128, None, 0,
                        None) == i4lib.I4_EALIGN
-    assert L.int4_gemm(None, fake, fake, None, fake, 0, 512, 16, 128, 128, None) == i4lib.I4_EINVAL
+    assert L.int4_gemm(None, fake, fake, None, fake, 0, 512, 16, 128, 128, None, 0, None) == i4lib.I4_EINVAL
+    assert L.int4_gemm(fake, fake, fake, None, fake, 0, 512, 16, 128, 128, ctypes.c_void_p((1 << 20) + 16), 1 << 20,
+                       None) == i4lib.I4_EALIGN
     odd = ctypes.c_void_p((1 << 20) + 4)
     assert L.int4_gemv(odd, fake, fake, None, fake, 0, 1, 16, 128, 128, None) == i4lib.I4_EALIGN
     assert L.paged_gqa_decode(fake, fake, fake, fake, fake, fake, 1, 28, 4, 64, 16, 4, 1.0, fake, 1 << 20,

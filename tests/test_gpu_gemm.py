@@ -19,23 +19,47 @@ pytestmark = pytest.mark.gpu
 TOL = 2e-3
 
 
-def run_gemm(i4, cuda, w, s, x, b=None, out_fp32=False):
+def run_gemm(i4, cuda, w, s, x, b=None, out_fp32=False, split=True):
+    """The GEMM with a split-K workspace (split=True: the launch configuration of batched decode and
+    prefill) or without one."""
     import torch
-    y = i4.int4_gemm(dev(w, cuda), dev(s, cuda), dev(x, cuda), None if b is None else dev(b, cuda), out_fp32=out_fp32)
+    M, K = x.shape
+    ws = None
+    if split:
+        ws = torch.zeros(max(i4.int4_gemm_ws_bytes(M, w.shape[0], K), 256), dtype=torch.uint8, device=cuda)
+    y = i4.int4_gemm(dev(w, cuda), dev(s, cuda), dev(x, cuda), None if b is None else dev(b, cuda), out_fp32=out_fp32,
+                     ws=ws)
     torch.cuda.synchronize()
     return y.cpu().numpy()
 
 
+@pytest.mark.parametrize("split", [True, False])
 @pytest.mark.parametrize("M,N,K", [(16, 256, 512), (20, 1000, 1024), (32, 4608, 3584), (64, 3584, 3584),
                                    (100, 384, 2048), (128, 640, 1024), (200, 512, 512), (300, 256, 2048),
                                    (512, 512, 3584)])
-def test_gemm_shapes_against_oracle(i4lib, cuda, M, N, K):
+def test_gemm_shapes_against_oracle(i4lib, cuda, M, N, K, split):
     w, s, x, b = synth.gemv_case(N, K, m=M, seed=M + N, bias=True)
-    got = run_gemm(i4lib, cuda, w, s, x, b)
+    got = run_gemm(i4lib, cuda, w, s, x, b, split=split)
     ref = oracle.f16(oracle.int4_linear(w, s, x, b))
     assert got.shape == (M, N)
     assert normwise_err(got, ref) <= TOL
     assert i4lib.device_error() == 0
+
+
+def test_gemm_weights_enter_exactly(i4lib, cuda):
+    """Scales whose products with the codes need more than fp16's 11 significant bits (so fp16(q * s) alone
+    would be off) and one-hot activations: y[m][n] = q[n][k_m] * s[n][k_m / 128] exactly, so the fp32 output
+    must equal the oracle's value bit for bit -- the two-term dequantisation holds every weight exactly."""
+    rng = np.random.default_rng(8)
+    M, N, K = 64, 256, 1024
+    w = rng.integers(0, 2**32, size=(N, K // 8), dtype=np.uint32)
+    s = rng.uniform(0.005, 0.02, size=(N, K // 128)).astype(np.float16)
+    ks = rng.choice(K, size=M, replace=False)
+    x = np.zeros((M, K), dtype=np.float16)
+    x[np.arange(M), ks] = 1.0
+    got = run_gemm(i4lib, cuda, w, s, x, out_fp32=True)
+    ref = oracle.int4_linear(w, s, x).astype(np.float32)
+    assert np.array_equal(got, ref)
 
 
 def test_gemm_fp32_output(i4lib, cuda):
