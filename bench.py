@@ -547,6 +547,63 @@ def run_gemv_batch(args):
     return 0
 
 
+def run_int8_ab(args):
+    """The INT8-activation A/B at the gate/up (K 3584, N 37888) and down (K 18944, N 3584) shapes, one vector:
+    the production tensor-core path (unpack 3), the exact CUDA-core fp16 unpack (0) and the int8-activation
+    dp4a variant (5), each L2-cold (a graph of (flush, GEMV) pairs minus the flushes), weight GB/s against the
+    measured HBM peak, and each one's normwise error against the oracle on 256 sampled rows."""
+    import numpy as np
+    import torch
+
+    import int4_weight_only_02_b200 as i4
+    import oracle
+    from int4_weight_only_02_b200 import synth
+    dev = torch.device("cuda", 0)
+    peak, peak_kind = measured_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    reps = 10
+    names = {3: "fp16 x, mma.sync (production)", 0: "fp16 x, exact CUDA-core unpack", 5: "int8 x, dp4a"}
+    for n, k in ((37888, 3584), (3584, 18944)):
+        w, s, x, _ = synth.gemv_case(n, k, seed=0)
+        wd, sd, xd = (torch.from_numpy(a.view(np.int32) if a.dtype == np.uint32 else a).to(dev) for a in (w, s, x))
+        y = torch.empty((1, n), dtype=torch.float16, device=dev)
+        rows = np.sort(np.random.default_rng(1).choice(n, size=256, replace=False))
+        ref = oracle.f16(oracle.int4_linear(w[rows], s[rows], x))
+        for unp in (3, 0, 5):
+            def graph_ms(with_gemv):
+                side = torch.cuda.Stream()
+                g = torch.cuda.CUDAGraph()
+                torch.cuda.synchronize()
+                with torch.cuda.stream(side):
+                    i4.int4_gemv(wd, sd, xd, y=y, unpack=unp, stream=side)
+                    with torch.cuda.graph(g, stream=side):
+                        for _ in range(reps):
+                            flush.add_(1)
+                            if with_gemv:
+                                i4.int4_gemv(wd, sd, xd, y=y, unpack=unp, stream=side)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                best = None
+                for _ in range(3):
+                    e0.record()
+                    g.replay()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    t = e0.elapsed_time(e1) / reps
+                    best = t if best is None else min(best, t)
+                return best
+
+            ms = graph_ms(True) - graph_ms(False)
+            err = float(np.max(np.abs(y.cpu().numpy()[0, rows].astype(np.float64) - ref[0])) /
+                        np.max(np.abs(ref[0].astype(np.float64))))
+            wbytes = n * (k // 2) + n * (k // 128) * 2
+            gbs = wbytes / (ms * 1e-3) / 1e9
+            print(json.dumps({"int8_ab": names[unp], "unpack": unp, "N": n, "K": k, "us": round(ms * 1e3, 2),
+                              "weight_GBs": round(gbs, 1), "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
+                              "normwise_err_vs_oracle": err, "device_error": i4.device_error()}), flush=True)
+    return 0
+
+
 def run_batched_decode(args):
     """B sequences of the 7B-shape decoder decoded together (one CUDA graph of library calls per step),
     each with its own 512-token prompt (teacher-forced, untimed) and page-table row; then K timed steps.
@@ -722,6 +779,8 @@ def main():
                     help="time to first token of a --prompt token prompt prefilled on the tcgen05 GEMM")
     ap.add_argument("--batched-decode", type=int, default=0,
                     help="decode this many sequences together (1..8) through the batched library calls")
+    ap.add_argument("--int8-ab", action="store_true",
+                    help="INT8-activation (dp4a) GEMV against the fp16 paths at the gate/up and down shapes")
     ap.add_argument("--gemv-batch", action="store_true",
                     help="INT4 GEMV at the gate/up shape for 1, 2, 4 and 8 vectors (weight GB/s)")
     args = ap.parse_args()
@@ -735,6 +794,8 @@ def main():
         return run_attention_sweep(args)
     if args.gemv_batch:
         return run_gemv_batch(args)
+    if args.int8_ab:
+        return run_int8_ab(args)
     if args.batched_decode:
         return run_batched_decode(args)
     if args.prefill:

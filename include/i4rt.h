@@ -390,6 +390,13 @@ I4_API int i4_device_error(int reset);
  * int4_gemv with an explicit unpack variant (as for "unpack") and a cap on the
  * number of CTAs (0 = none; any cap selects the register-streaming kernel
  * instead of the bulk-copy pipelined one); for tests and benchmarks.
+ * unpack 5 is the INT8-activation variant, the alternative the pages' lesson on
+ * byte permutes against __dp4a describes: x is quantised to int8 per 128-group
+ * (scale max|x| / 127, round to nearest), the nibbles become offset-binary
+ * bytes, dp4a sums the products with an exact -8 * sum(x) correction, and the
+ * group's integer sum is scaled by s_w * s_x in fp32. Its result carries the
+ * int8 rounding of x (it is not the INT4 weight-only product); M == 1 and
+ * K % 512 == 0 only (the bulk-copy streaming kernel, plain fp16/fp32 output).
  */
 I4_API int i4_int4_gemv_variant(const uint32_t *w, const uint16_t *scales, const uint16_t *x, const uint16_t *bias,
                                 void *y, int y_is_fp32, int M, int N, int K, int unpack, int max_ctas, void *stream);

@@ -177,6 +177,7 @@ int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool p
     if (unp == UNPACK_AUTO) unp = a.M <= 8 ? UNPACK_MMA : UNPACK_EXACT;
     StreamGeom geo;
     if (max_ctas == 0 && stream_geometry(epi, a, geo, unp)) return launch_gemv_stream(pro, epi, a, geo, stream, pdl, unp);
+    if (unp == UNPACK_DP4A) return fail(I4_EUNSUPPORTED, "int8-activation gemv: shape outside the streaming kernel");
     if (max_ctas == 0 && unp == UNPACK_MMA && stream_geometry(epi, a, geo, UNPACK_SUBNORMAL))
         return launch_gemv_stream(pro, epi, a, geo, stream, pdl, UNPACK_SUBNORMAL);  // rows too long for 16-row tiles
     if (unp == UNPACK_MAGIC32 || unp == UNPACK_MMA) unp = UNPACK_SUBNORMAL;  // register kernel: fp16 unpacks only
@@ -239,7 +240,9 @@ extern "C" int int4_gemv(const uint32_t *w, const uint16_t *scales, const uint16
 extern "C" int i4_int4_gemv_variant(const uint32_t *w, const uint16_t *scales, const uint16_t *x,
                                     const uint16_t *bias, void *y, int y_is_fp32, int M, int N, int K, int unpack,
                                     int max_ctas, void *stream) {
-    if (unpack < UNPACK_EXACT || unpack > UNPACK_AUTO) return fail(I4_EINVAL, "unknown unpack variant");
+    if (unpack < UNPACK_EXACT || unpack > UNPACK_DP4A) return fail(I4_EINVAL, "unknown unpack variant");
+    if (unpack == UNPACK_DP4A && (M != 1 || max_ctas != 0 || K % 512 != 0))
+        return fail(I4_EUNSUPPORTED, "int8-activation gemv: one vector, K %% 512 == 0, the streaming kernel");
     return gemv_entry(w, scales, x, bias, y, y_is_fp32, M, N, K, 128, unpack, max_ctas, (cudaStream_t)stream);
 }
 

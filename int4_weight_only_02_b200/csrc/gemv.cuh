@@ -12,7 +12,11 @@ enum GemvPrologue : int { PRO_PLAIN = 0, PRO_RMSNORM = 1, PRO_EMBED = 2 };
 enum GemvEpilogue : int { EPI_F16 = 0, EPI_F32 = 1, EPI_RESID = 2, EPI_ROPE_KV = 3, EPI_SILU = 4, EPI_ARGMAX = 5 };
 // UNPACK_AUTO picks per launch: the tensor-core kernels (single-vector, or batched for M <= 8 with rows of
 // up to 4096 weights; the fastest measured), else the exact CUDA-core unpack.
-enum GemvUnpack : int { UNPACK_EXACT = 0, UNPACK_SUBNORMAL = 1, UNPACK_MAGIC32 = 2, UNPACK_MMA = 3, UNPACK_AUTO = 4 };
+// UNPACK_DP4A is the INT8-activation variant (x quantised to int8 per 128-group, dp4a products); it changes
+// the arithmetic, so it is selected only explicitly (i4_int4_gemv_variant), for comparison.
+enum GemvUnpack : int {
+    UNPACK_EXACT = 0, UNPACK_SUBNORMAL = 1, UNPACK_MAGIC32 = 2, UNPACK_MMA = 3, UNPACK_AUTO = 4, UNPACK_DP4A = 5
+};
 
 struct GemvArgs {
     const uint32_t *w;

@@ -297,11 +297,74 @@ __device__ __forceinline__ void half_acc_f32(uint2 w, const float4 *x4, float s,
     r.hi = acc.y;
 }
 
+// INT8-activation variant: x quantised to int8 per 128-group (scale sx_g = max|x_g| / 127, round to
+// nearest), the weight nibbles turned into offset-binary bytes u = q + 8 with one LOP3 (low nibbles) or a
+// shift and a LOP3 (high nibbles), four dp4a per 16 weights against the int8 x bytes in the same order, and
+// the exact integer correction - 8 * sum(x_q); the integer sum of the half-chunk is then scaled by
+// s_w * sx_g in fp32. xq = (x0,x2,x4,x6) (x1,x3,x5,x7) (x8,x10,x12,x14) (x9,x11,x13,x15) of the half-chunk.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ void half_acc_dp4a(uint2 w, const uint4 &xq, int sq, float s_w_sx, RowAcc &r) {
+    const uint32_t la = lop3_and_xor(w.x, 0x0F0F0F0Fu, 0x08080808u);
+    const uint32_t ha = lop3_and_xor(w.x >> 4, 0x0F0F0F0Fu, 0x08080808u);
+    const uint32_t lb = lop3_and_xor(w.y, 0x0F0F0F0Fu, 0x08080808u);
+    const uint32_t hb = lop3_and_xor(w.y >> 4, 0x0F0F0F0Fu, 0x08080808u);
+    int acc = dp4a_us(la, xq.x, -8 * sq);
+    acc = dp4a_us(ha, xq.y, acc);
+    acc = dp4a_us(lb, xq.z, acc);
+    acc = dp4a_us(hb, xq.w, acc);
+    r.lo = fmaf((float)acc, s_w_sx, r.lo);
+}
+
 template <int UNP>
 __device__ __forceinline__ float row_value(const RowAcc &r) {
     if constexpr (UNP == UNPACK_MAGIC32) return r.lo + r.hi;
-    if constexpr (UNP == UNPACK_EXACT) return r.lo;
+    if constexpr (UNP == UNPACK_EXACT || UNP == UNPACK_DP4A) return r.lo;
     return fmaf(r.hi, 0.0625f, r.lo) * 16777216.0f - 8.0f * r.cx;
+}
+
+// INT8 stage: x (after the prologue) quantised per 128-group. xq[h] holds half-chunk h's 16 values as int8 in
+// the dp4a order above, sq[h] their integer sum, scx[g] the group's scale; tmp holds K fp16 values.
+template <int PRO, class Group>
+__device__ __forceinline__ void stage_x_int8(const GemvArgs &a, uint4 *xq, int *sq, float *scx, uint16_t *tmp,
+                                             float *red, const Group &grp) {
+    const int K = a.K, groups = K >> 7, nhr = K >> 4;
+    for_each_x_word<PRO>(a, red, grp, [&](int c, uint4 v) { reinterpret_cast<uint4 *>(tmp)[c] = v; });
+    grp.sync();
+    // group scales: a warp per group
+    const int warp = grp.tid() >> 5, lane = grp.tid() & 31, nw = grp.size() >> 5;
+    for (int g = warp; g < groups; g += nw) {
+        float m = 0.f;
+        for (int i = lane; i < 128; i += 32) m = fmaxf(m, fabsf(half_bits_to_float(tmp[g * 128 + i])));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        if (lane == 0) scx[g] = m > 0.f ? m / 127.0f : 1.0f;
+    }
+    grp.sync();
+    for (int h = grp.tid(); h < nhr; h += grp.size()) {
+        const float inv = 1.0f / scx[h >> 3];
+        int q[16], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            int v = __float2int_rn(half_bits_to_float(tmp[16 * h + i]) * inv);
+            v = v > 127 ? 127 : (v < -127 ? -127 : v);
+            q[i] = v;
+            sum += v;
+        }
+        auto pack = [&](int o) {  // bytes x_o, x_{o+2}, x_{o+4}, x_{o+6}
+            return (uint32_t)(q[o] & 0xFF) | ((uint32_t)(q[o + 2] & 0xFF) << 8) | ((uint32_t)(q[o + 4] & 0xFF) << 16) |
+                   ((uint32_t)(q[o + 6] & 0xFF) << 24);
+        };
+        xq[h] = make_uint4(pack(0), pack(1), pack(8), pack(9));
+        sq[h] = sum;
+    }
 }
 
 // Stage x (MR vectors of K fp16) into shared memory, pair-permuted:

@@ -96,6 +96,11 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_stream_kernel(const Ge
     uint4 *xo = xe + nhr;
     float *sxh = reinterpret_cast<float *>(xo + nhr);
     const float4 *xf = reinterpret_cast<const float4 *>(xe);  // fp32 unpack: K floats in place of xe/xo/sxh
+    // INT8 activations: xq [K/16] uint4, sq [K/16] int, scx [K/128] float, then K fp16 of staging space
+    uint4 *xq = xe;
+    int *sq = reinterpret_cast<int *>(xq + nhr);
+    float *scx = reinterpret_cast<float *>(sq + nhr);
+    uint16_t *xtmp = reinterpret_cast<uint16_t *>(scx + (K >> 7));
     // balanced contiguous ranges: tile counts of any two CTAs differ by at most one
     const int t_begin = (int)(((long long)blockIdx.x * geo.tiles) / gridDim.x);
     const int t_end = (int)(((long long)(blockIdx.x + 1) * geo.tiles) / gridDim.x);
@@ -130,6 +135,8 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_stream_kernel(const Ge
         grid_dep_wait();
         if constexpr (UNP == UNPACK_MAGIC32)
             stage_x_f32<PRO>(a, reinterpret_cast<float4 *>(xe), red, grp);
+        else if constexpr (UNP == UNPACK_DP4A)
+            stage_x_int8<PRO>(a, xq, sq, scx, xtmp, red, grp);
         else
             stage_x_halves<PRO, UNP>(a, xe, xo, sxh, red, grp);
         grp.sync();
@@ -145,9 +152,15 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_stream_kernel(const Ge
             for (int i = 0; i < kMaxHalvesPerLane; ++i) {
                 if (UNP != UNPACK_MAGIC32 && i < nh) {
                     const int h = lane + 32 * i;
-                    x0[i] = xe[h];
-                    x1[i] = xo[h];
-                    sx[i] = (UNP == UNPACK_SUBNORMAL) ? sxh[h] : 0.f;
+                    if constexpr (UNP == UNPACK_DP4A) {  // x0: int8 x, sx: its group scale, x1.x: its integer sum
+                        x0[i] = xq[h];
+                        sx[i] = scx[h >> 3];
+                        x1[i] = make_uint4((uint32_t)sq[h], 0u, 0u, 0u);
+                    } else {
+                        x0[i] = xe[h];
+                        x1[i] = xo[h];
+                        sx[i] = (UNP == UNPACK_SUBNORMAL) ? sxh[h] : 0.f;
+                    }
                 }
             }
             const int tra = kPaired<EPI> ? warp : 2 * warp, trb = kPaired<EPI> ? warp + 8 : 2 * warp + 1;
@@ -177,6 +190,9 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_stream_kernel(const Ge
                                 for (int e = 0; e < 4; ++e) x4[e] = xf[4 * h + e];
                                 half_acc_f32(wa[h], x4, half_bits_to_float(sa[h >> 3]), ra);
                                 half_acc_f32(wb[h], x4, half_bits_to_float(sb[h >> 3]), rb);
+                            } else if constexpr (UNP == UNPACK_DP4A) {
+                                half_acc_dp4a(wa[h], x0[k], (int)x1[k].x, half_bits_to_float(sa[h >> 3]) * sx[k], ra);
+                                half_acc_dp4a(wb[h], x0[k], (int)x1[k].x, half_bits_to_float(sb[h >> 3]) * sx[k], rb);
                             } else {
                                 half_acc<UNP>(wa[h], x0[k], x1[k], half_bits_to_float(sa[h >> 3]), sx[k], ra);
                                 half_acc<UNP>(wb[h], x0[k], x1[k], half_bits_to_float(sb[h >> 3]), sx[k], rb);
@@ -218,6 +234,11 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_stream_kernel(const Ge
                             for (int e = 0; e < 4; ++e) x4[e] = xf[4 * h + e];
                             half_acc_f32(w0[h], x4, half_bits_to_float(s0[h >> 3]), r0);
                             half_acc_f32(w1[h], x4, half_bits_to_float(s1[h >> 3]), r1);
+                        } else if constexpr (UNP == UNPACK_DP4A) {
+                            const uint4 q4 = xq[h];
+                            const float g = scx[h >> 3];
+                            half_acc_dp4a(w0[h], q4, sq[h], half_bits_to_float(s0[h >> 3]) * g, r0);
+                            half_acc_dp4a(w1[h], q4, sq[h], half_bits_to_float(s1[h >> 3]) * g, r1);
                         } else {
                             const uint4 e = xe[h], o = xo[h];
                             const float sxv = (UNP == UNPACK_SUBNORMAL) ? sxh[h] : 0.f;
@@ -681,7 +702,9 @@ bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp) {
     g.R = R;
     g.stage_bytes = (int)(((R * (wrow + srow)) + 127) / 128 * 128);
     const long long xs_bytes =
-        unp == UNPACK_MAGIC32 ? (long long)a.K * 4 : (long long)a.K * 2 + (long long)(a.K / 16) * 4;
+        unp == UNPACK_MAGIC32 ? (long long)a.K * 4
+        : unp == UNPACK_DP4A  ? (long long)a.K + (long long)(a.K / 16) * 4 + (long long)(a.K / 128) * 4 + (long long)a.K * 2
+                              : (long long)a.K * 2 + (long long)(a.K / 16) * 4;
     long long room = g_stream_smem_budget - xs_bytes;
     int stages = (int)(room / g.stage_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
@@ -780,6 +803,12 @@ template <int PRO, int EPI>
 static int launch_stream_u(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl, int unp) {
     if (unp == UNPACK_MMA) return launch_mma_t<PRO, EPI>(a, geo, stream, pdl);
     if (unp == UNPACK_MAGIC32) return launch_stream_r<PRO, EPI, UNPACK_MAGIC32>(a, geo, stream, pdl);
+    if (unp == UNPACK_DP4A) {
+        if constexpr (PRO == PRO_PLAIN && (EPI == EPI_F16 || EPI == EPI_F32))
+            return launch_stream_r<PRO, EPI, UNPACK_DP4A>(a, geo, stream, pdl);
+        else
+            return fail(I4_EUNSUPPORTED, "int8-activation gemv: plain x and fp16/fp32 output only");
+    }
     if (unp == UNPACK_SUBNORMAL) return launch_stream_r<PRO, EPI, UNPACK_SUBNORMAL>(a, geo, stream, pdl);
     return launch_stream_r<PRO, EPI, UNPACK_EXACT>(a, geo, stream, pdl);
 }

@@ -116,8 +116,10 @@ def test_bad_arguments_raise(i4lib, cuda):
     xd = dev(x, cuda)
     with pytest.raises(i4lib.I4Error):
         i4lib.int4_gemv(wd, sd, xd, group=64)
-    with pytest.raises(i4lib.I4Error):
-        i4lib.int4_gemv(wd, sd, torch.zeros((9, 256), dtype=torch.float16, device=cuda))
+    with pytest.raises(i4lib.I4Error):  # K not a multiple of the group
+        i4lib.int4_gemv(wd[:, :12], sd, torch.zeros((2, 96), dtype=torch.float16, device=cuda))
+    with pytest.raises(i4lib.I4Error):  # the int8-activation variant takes one vector only
+        i4lib.int4_gemv(wd, sd, torch.zeros((2, 256), dtype=torch.float16, device=cuda), unpack=5)
 
 
 @pytest.mark.parametrize("n,k", [(3584, 18944), (64, 4608), (30, 8192), (6, 2560), (14, 1536)])
