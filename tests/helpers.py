@@ -14,12 +14,22 @@ def dev(a, device):
     return to_device(np.asarray(a), device)
 
 
-# Greedy-decode tie bound of the 28-layer 7B-shape decoder, derived on the oracle
-# alone (test_oracle_sensitivity.py): fp32 sums round about 1 % of fp16 stores
-# differently from fp64 sums; injecting such +-1-ulp flips at a 1 % rate into the
-# oracle moves the last-token logits by ~0.06-0.08 RMS (up to ~0.4) after a
-# 64-128 token context, so a top-2 gap below 3 * sqrt(2) * 0.07 ~= 0.3 is a tie
-# that neither implementation can be held to.
-FLIP_RATE = 0.01
-TIE_GAP = 0.3
-LOGIT_NOISE_MAX = 0.4
+# Greedy-decode tie bound of the 28-layer 7B-shape decoder. The per-layer
+# teacher-forced comparison (test_gpu_layer_parity.py) measures how often the
+# GPU's fp16 stores differ from the oracle's: at most 1.7 % per tensor
+# (attention output of layer 27) where each element rounds on its own. One
+# tensor reads higher, silu(gate)*up of layer 13 at 21 %, and it is not
+# independent noise: there a single element of the RMSNorm output (1 of 3584)
+# rounds to the other fp16 neighbour, every gate/up dot product moves by the
+# same fraction of an ulp, and many products that sat near a rounding boundary
+# cross it together (the fused kernel gives the same bits as the stand-alone
+# RMSNorm, GEMV and SiLU kernels chained). A one-ulp change of one input
+# element is the case the sensitivity test measures separately (<= 0.075).
+# Injecting independent +-1-ulp flips at 1.7 % into every fp16 store of the
+# oracle (test_oracle_sensitivity.py) moves the last-token logits after a
+# 64-token prompt by 0.076-0.079 RMS and at most 0.42 (seeds 200, 201), so a
+# top-2 gap below 3 * sqrt(2) * 0.079 ~= 0.34 is a tie neither side can be held
+# to, and a first-step logit within 0.45 of the oracle's is inside the noise.
+FLIP_RATE = 0.017
+TIE_GAP = 0.35
+LOGIT_NOISE_MAX = 0.45

@@ -34,7 +34,7 @@ import pytest
 
 import oracle
 from int4_weight_only_02_b200 import synth
-from helpers import normwise_err
+from helpers import FLIP_RATE, normwise_err
 
 pytestmark = pytest.mark.gpu
 
@@ -228,6 +228,13 @@ def test_each_kernel_teacher_forced(i4lib, cuda, oracle_run, gpu_step):
         print(f"layer {r['layer']:>5} {r['tensor']:<24} normwise {r['normwise']:.2e} "
               + (f"fp16 mismatch {r['fp16_mismatch']:.4f}" if r["fp16_mismatch"] is not None else ""))
     print(f"worst fp16 mismatch rate {worst:.4f}")
+    # The tie bound assumes independent one-ulp flips at FLIP_RATE at most. Every tensor whose fp16
+    # elements round independently stays there; silu(gate)*up may read higher because one RMSNorm
+    # output element that rounds to the other neighbour moves all gate/up products together (layer 13:
+    # 21 % of the stores, normwise 4.6e-4; the same bits come out of the stand-alone kernels chained).
+    for r in rep.rows:
+        if r["fp16_mismatch"] is not None and r["tensor"] != "silu(gate)*up":
+            assert r["fp16_mismatch"] <= FLIP_RATE, r
     path = os.environ.get("I4_PARITY_REPORT")
     if path:
         path = path.replace(".json", "_persistent.json" if graph.persistent else "_per_kernel.json")

@@ -16,7 +16,7 @@ import pytest
 import oracle
 import oracle.model as oracle_model
 from int4_weight_only_02_b200 import synth
-from helpers import FLIP_RATE, TIE_GAP
+from helpers import FLIP_RATE, LOGIT_NOISE_MAX, TIE_GAP
 
 LOGIT_NOISE_ONE_ULP = 0.075  # largest single-logit change from one ulp in one input element (measured 0.073)
 
@@ -57,12 +57,14 @@ def _flipping_f16(rng, rate):
 
 
 @pytest.mark.slow
-def test_one_percent_fp16_flips_set_the_greedy_tie_bound(monkeypatch):
-    """Noise model of fp32-vs-fp64 accumulation: 1 % of every stored fp16 tensor one ulp off.
+def test_measured_flip_rate_sets_the_greedy_tie_bound(monkeypatch):
+    """Noise model of fp32-vs-fp64 accumulation: FLIP_RATE (the largest independent fp16
+    mismatch rate measured per tensor on the GPU, 1.7 %) of every stored fp16 tensor one ulp off.
 
     The last-token logits after a 64-token prompt move by several hundredths
     RMS; three standard deviations of a top-2 gap difference must stay within
-    the tie bound the GPU decode test uses."""
+    the tie bound the GPU decode test uses, and the largest logit change within
+    the first-step noise ceiling."""
     shape = synth.QWEN7B
     layers = [synth.layer_weights(shape, i, 0) for i in range(shape.layers)]
     glob = synth.global_weights(shape, 0)
@@ -76,3 +78,4 @@ def test_one_percent_fp16_flips_set_the_greedy_tie_bound(monkeypatch):
     rms = float(np.sqrt(np.mean(d * d)))
     assert rms > 0.01
     assert 3 * np.sqrt(2) * rms <= TIE_GAP, rms
+    assert np.max(np.abs(d)) <= LOGIT_NOISE_MAX, np.max(np.abs(d))
