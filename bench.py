@@ -329,6 +329,9 @@ def run_profile_kernel(args):
         i4.set_option("unpack", args.unpack)
     if args.gemv_ctas is not None:
         i4.set_option("gemv_ctas_per_sm", args.gemv_ctas)
+    if args.gemv_prex is not None:
+        i4.set_option("gemv_prex", args.gemv_prex)
+
     if args.l2_prefetch is not None:
         i4.set_option("l2_prefetch", args.l2_prefetch)
     if args.persistent is not None:
@@ -760,6 +763,8 @@ def main():
     ap.add_argument("--pdl", type=int, default=None, help="override programmatic dependent launch (0/1)")
     ap.add_argument("--unpack", type=int, default=None, help="override the GEMV unpack variant (0..4, 4 = per shape)")
     ap.add_argument("--gemv-ctas", type=int, default=None, help="override the GEMV CTAs per SM (1 or 2)")
+    ap.add_argument("--gemv-prex", type=int, default=None,
+                    help="override the weight stages a GEMV copies before its loads of x are issued (0..8)")
     ap.add_argument("--l2-prefetch", type=int, default=None, help="override the next-GEMV L2 prefetch (0/1)")
     ap.add_argument("--l2-ahead", type=int, default=None,
                     help="override the tiles each CTA of the persistent step prefetches into L2 ahead (0..64)")
@@ -826,6 +831,9 @@ def main():
         i4.set_option("unpack", args.unpack)
     if args.gemv_ctas is not None:
         i4.set_option("gemv_ctas_per_sm", args.gemv_ctas)
+    if args.gemv_prex is not None:
+        i4.set_option("gemv_prex", args.gemv_prex)
+
     if args.l2_prefetch is not None:
         i4.set_option("l2_prefetch", args.l2_prefetch)
     if args.persistent is not None:

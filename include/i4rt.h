@@ -365,6 +365,9 @@ I4_API int decode_step_buffer_copy(i4_graph *g, int which, void *dev, size_t byt
  *            (M == 1, K % 512 == 0, 16-byte aligned w and scales), default 1;
  *   "stream_smem_kb" 32..227: shared memory budget of that kernel's ring;
  *   "gemv_ctas_per_sm" 1/2 (default 2): CTAs per SM of the pipelined GEMV grids;
+ *   "gemv_prex" 0..8 (default 1): weight stages the tensor-core GEMV copies
+ *            before its loads of x are issued (the rest follow them, so x does
+ *            not queue behind a full ring of weight copies);
  *   "l2_ahead" 0..64 (default 8): tiles of its own weight stream each CTA of a
  *            persistent step prefetches into L2 ahead of its shared-memory ring;
  *   "trace"  0/1 (default 0): persistent steps created afterwards record phase

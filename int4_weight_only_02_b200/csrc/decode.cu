@@ -32,6 +32,7 @@ extern bool g_l2_prefetch;
 bool g_dry_run = false;
 bool g_pdl = true;
 bool g_l2_prefetch = false;
+
 bool g_persistent = false;
 bool g_trace = false;
 int g_l2_ahead = 8;
@@ -50,6 +51,7 @@ struct i4_graph {
     float2 *rope_cs = nullptr;
     unsigned long long *best = nullptr;
     unsigned *arrive = nullptr;
+    unsigned *sched = nullptr;  // per kernel of the step: the counter pair of a GEMV's dynamic tile schedule
     char *attn_ws = nullptr;
     AttnWs attn_layout = {};
     cudaStream_t cap = nullptr;
@@ -126,6 +128,7 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
             a.max_ctx = d.max_ctx;
             a.status = g->seq.status;
             prefetch(a, L.w_o, L.s_o, H, d.n_q_heads * D);
+            a.sched = nullptr;  // fixed ranges: measured faster here
             if (!skip() && (st_ = launch_gemv(l == 0 ? PRO_EMBED : PRO_RMSNORM, EPI_ROPE_KV, a, st, pdl(), g->unpack, 0))) return st_;
             ++n;
         }
@@ -163,6 +166,7 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
             a.x = g->attn;
             a.y = g->resid;
             prefetch(a, L.w_gate_up, L.s_gate_up, 2 * I, H);
+            a.sched = nullptr;  // fixed ranges: measured faster here
             if (!skip() && (st_ = launch_gemv(PRO_PLAIN, EPI_RESID, a, st, pdl(), g->unpack, 0))) return st_;
             ++n;
         }
@@ -179,6 +183,7 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
             a.y = g->mlp;
             a.inter = I;
             prefetch(a, L.w_down, L.s_down, H, I);
+            a.sched = nullptr;  // fixed ranges: measured faster here
             if (!skip() && (st_ = launch_gemv(PRO_RMSNORM, EPI_SILU, a, st, pdl(), g->unpack, 0))) return st_;
             ++n;
         }
@@ -195,6 +200,7 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
                 prefetch(a, g->layers[l + 1].w_qkv, g->layers[l + 1].s_qkv, nqkv, H);
             else
                 prefetch(a, g->w.w_lm, g->w.s_lm, d.vocab, H);
+            a.sched = g->sched ? g->sched + 2 * n : nullptr;  // dynamic tiles: measured faster here
             if (!skip() && (st_ = launch_gemv(PRO_PLAIN, EPI_RESID, a, st, pdl(), g->unpack, 0))) return st_;
             ++n;
         }
@@ -220,7 +226,8 @@ static int enqueue_step(i4_graph *g, cudaStream_t st, int *count, int only = -1)
         a.history = g->seq.history;
         a.max_ctx = d.max_ctx;
         a.status = g->seq.status;
-        if (!skip() && (st_ = launch_gemv(PRO_RMSNORM, EPI_ARGMAX, a, st, pdl(), g->unpack, 0))) return st_;
+        a.sched = g->sched ? g->sched + 2 * n : nullptr;  // dynamic tiles: measured faster here
+            if (!skip() && (st_ = launch_gemv(PRO_RMSNORM, EPI_ARGMAX, a, st, pdl(), g->unpack, 0))) return st_;
         ++n;
     }
     if (count) *count = n;
@@ -317,6 +324,7 @@ extern "C" int decode_step_graph_create(const i4_model_desc *desc, const i4_mode
     const size_t o_mlp = off; off += a256((size_t)desc->intermediate * 2);
     const size_t o_rope = off; off += a256((size_t)desc->max_ctx * (D / 2) * sizeof(float2));
     const size_t o_best = off; off += 256;
+    const size_t o_sched = off; off += a256((size_t)(5 * desc->n_layers + 1) * 2 * sizeof(unsigned));
     const size_t o_attn_ws = off; off += a256(g->attn_layout.bytes);
     g->n_phases = 5 * desc->n_layers + 1;
     if (g_persistent) g->plan = persist_plan(*desc);
@@ -337,6 +345,7 @@ extern "C" int decode_step_graph_create(const i4_model_desc *desc, const i4_mode
     g->rope_cs = reinterpret_cast<float2 *>(g->ws + o_rope);
     g->best = reinterpret_cast<unsigned long long *>(g->ws + o_best);
     g->arrive = reinterpret_cast<unsigned *>(g->ws + o_best + 8);
+    g->sched = reinterpret_cast<unsigned *>(g->ws + o_sched);
     g->attn_ws = g->ws + o_attn_ws;
 
     std::vector<PPhase> phases;
@@ -528,6 +537,11 @@ extern "C" int i4_set_option(const char *name, int value) {
     }
     if (n == "l2_prefetch") {
         g_l2_prefetch = value != 0;
+        return I4_OK;
+    }
+    if (n == "gemv_prex") {
+        if (value < 0 || value > 8) return fail(I4_EINVAL, "gemv_prex must be in [0, 8]");
+        set_stream_prex(value);
         return I4_OK;
     }
     if (n == "gemv_ctas_per_sm") {

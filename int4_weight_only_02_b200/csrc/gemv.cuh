@@ -50,6 +50,9 @@ struct GemvArgs {
     // the CTAs, issued once the ring is first filled); null pointers = none
     const void *pf_a, *pf_b;
     size_t pf_a_bytes, pf_b_bytes;
+    // tensor-core GEMV: two zeroed counters of a dynamic tile schedule, owned by this launch until it
+    // completes (left zeroed again); null = each CTA takes a fixed contiguous range of tiles
+    unsigned *sched;
 };
 
 size_t gemv_smem_bytes(int K, int mr, int unp);
@@ -61,6 +64,7 @@ struct StreamGeom {
     int stages;         // ring depth
     int tiles, tiles_per_cta, grid;
     int smem;           // dynamic shared memory bytes
+    int prex;           // tensor-core consumer: stages copied before the loads of x are issued
 };
 // False when the shape or alignment does not fit the streaming kernel.
 bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp);
@@ -68,6 +72,7 @@ int launch_gemv_stream(int pro, int epi, const GemvArgs &a, const StreamGeom &ge
                        int unp);
 void set_stream_options(int enabled, int smem_kb);
 void set_stream_ctas_per_sm(int n);
+void set_stream_prex(int n);
 // unp < 0 selects the library default; max_ctas <= 0 means no cap.
 int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool pdl, int unp, int max_ctas);
 

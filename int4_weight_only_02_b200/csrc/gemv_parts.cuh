@@ -125,6 +125,17 @@ struct NamedGroup {
     __device__ __forceinline__ void sync() const { asm volatile("bar.sync 1, %0;" ::"n"(COUNT) : "memory"); }
 };
 
+// Named barrier 1 over the 256 consumer threads that also ANDs a predicate across them.
+__device__ __forceinline__ bool bar1_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+
 template <class Group>
 __device__ __forceinline__ float group_sum(float v, float *red, const Group &g) {
     v = warp_sum(v);

@@ -34,6 +34,8 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kStreamThreads = kConsumers + 32;  // warp 0 produces
 constexpr int kMaxStages = 8;
+constexpr int kWin = 8;  // tiles per epilogue window of the tensor-core consumer
+constexpr int kStaticTiles = 2;  // tiles per CTA assigned before the shared counter takes over
 
 __device__ int g_device_error = 0;
 
@@ -332,141 +334,348 @@ __device__ __forceinline__ void prefetch_share(const void *base, size_t bytes) {
     }
 }
 
-template <int PRO, class Group>
-__device__ __forceinline__ void stage_x_tc(const GemvArgs &a, uint4 *xt, float *sx8, float *red, const Group &grp) {
-    const int nb = tc_blocks(a.K), groups = a.K >> 7;
+// RMSNorm prologues: gamma words held in registers from before the dependency wait (gamma does not
+// depend on the previous kernel), for rows of up to kXRegWords * 8 * 256 = 4096 weights.
+constexpr int kXRegWords = 2;
+
+// Word c of x into the lane-order layout, and the sum of its 128-weight group into sx8 (times 8):
+// the 16 words of a group sit on 16 consecutive lanes of one warp (c = thread + 256 k, K % 128 == 0),
+// so four xor-shuffles give the group sum. Every lane of the warp calls it (v = 0 and no store past K).
+__device__ __forceinline__ void stage_word_tc(uint4 *xt, float *sx8, int c, int nwords, uint4 v) {
+    float t = 0.f;
+    if (c < nwords) {
+        const int b = c >> 7, l = (c & 127) >> 2, w = c & 3;
+        const uint4 pp = permute_pairs(v);  // (x0,x4) (x1,x5) (x2,x6) (x3,x7)
+        xt[(b * 4 + w) * 32 + l] = make_uint4(pp.x, pp.z, pp.y, pp.w);
+        const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[q]));
+            t += f.x + f.y;
+        }
+    }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if ((threadIdx.x & 15) == 0 && c < nwords) sx8[c >> 4] = 8.0f * t;
+}
+
+// fp16(r / sqrt(mean(r^2) + eps) * gamma) of one word (fp32 math, the formula of every RMSNorm here)
+__device__ __forceinline__ uint4 rmsnorm_word(uint4 rv, uint4 gv, float inv) {
+    const uint32_t r[4] = {rv.x, rv.y, rv.z, rv.w}, g[4] = {gv.x, gv.y, gv.z, gv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const float2 fr = __half22float2(*reinterpret_cast<const __half2 *>(&r[t]));
+        const float2 fg = __half22float2(*reinterpret_cast<const __half2 *>(&g[t]));
+        const __half2 h = __floats2half2_rn(fr.x * inv * fg.x, fr.y * inv * fg.y);
+        o[t] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ float sumsq_word(uint4 rv, float ss) {
+    const uint32_t r[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&r[t]));
+        ss = fmaf(f.x, f.x, ss);
+        ss = fmaf(f.y, f.y, ss);
+    }
+    return ss;
+}
+
+// Stage x (plain, RMSNorm of the residual row, or RMSNorm of the embedding row) in lane order with
+// its group sums. Thread t owns words t, t + 256, ...; loads are issued together before any use, so
+// one memory latency covers the row (the weight copies of this kernel are already queued ahead of it).
+template <int PRO, int LB, class Group>
+__device__ __forceinline__ void stage_x_tc(const GemvArgs &a, uint4 *xt, float *sx8, float *red, const Group &grp,
+                                           const uint4 (&gpre)[kXRegWords], uint64_t *xbar) {
+    // tells the producer that this warp's loads of x are issued (the weight copies it holds back go after them)
+    auto issued = [&]() {
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(xbar);
+    };
+    const int K = a.K, nwords = K >> 3, nb = tc_blocks(K), T = grp.size(), tid = grp.tid();
+    const int rounds = (nwords + T - 1) / T;
     // zero the padding past K (lanes of a partial last block read it)
-    for (int i = (a.K >> 3) + grp.tid(); i < nb * 128; i += grp.size()) {
+    for (int i = nwords + tid; i < nb * 128; i += T) {
         const int b = i >> 7, l = (i & 127) >> 2, w = i & 3;
         xt[(b * 4 + w) * 32 + l] = make_uint4(0u, 0u, 0u, 0u);
     }
-    for_each_x_word<PRO>(a, red, grp, [&](int wd, uint4 v) {
-        const int b = wd >> 7, l = (wd & 127) >> 2, w = wd & 3;
-        const uint4 pp = permute_pairs(v);  // (x0,x4) (x1,x5) (x2,x6) (x3,x7)
-        xt[(b * 4 + w) * 32 + l] = make_uint4(pp.x, pp.z, pp.y, pp.w);
-    });
-    grp.sync();
-    for (int j = grp.tid(); j < groups; j += grp.size()) {
-        const int b = j >> 3, g = j & 7;
-        float t = 0.f;
-        for (int w = 0; w < 4; ++w)
-            for (int c = 0; c < 4; ++c) {
-                const uint4 e = xt[(b * 4 + w) * 32 + 4 * g + c];
-                const uint32_t v[4] = {e.x, e.y, e.z, e.w};
-                for (int q = 0; q < 4; ++q) {
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&v[q]));
-                    t += f.x + f.y;
-                }
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (PRO == PRO_PLAIN) {
+        for (int k0 = 0; k0 < rounds; k0 += LB) {  // LB loads in flight per thread
+            uint4 v[LB];
+#pragma unroll
+            for (int u = 0; u < LB; ++u) {
+                const int c = tid + T * (k0 + u);
+                v[u] = c < nwords ? *reinterpret_cast<const uint4 *>(a.x + 8 * c) : zero;
             }
-        sx8[j] = 8.0f * t;
+            if (k0 == 0) issued();
+#pragma unroll
+            for (int u = 0; u < LB; ++u)
+                if (k0 + u < rounds) stage_word_tc(xt, sx8, tid + T * (k0 + u), nwords, v[u]);
+        }
+    } else {
+        const uint16_t *src = a.x;
+        if constexpr (PRO == PRO_EMBED) {
+            int tok = *a.token;
+            tok = tok < 0 ? 0 : (tok >= a.vocab ? a.vocab - 1 : tok);
+            src = a.x + (size_t)tok * K;
+        }
+        if (rounds <= kXRegWords) {
+            uint4 r[kXRegWords];
+            float ss = 0.f;
+#pragma unroll
+            for (int u = 0; u < kXRegWords; ++u) {
+                const int c = tid + T * u;
+                r[u] = c < nwords ? *reinterpret_cast<const uint4 *>(src + 8 * c) : zero;
+            }
+            issued();
+#pragma unroll
+            for (int u = 0; u < kXRegWords; ++u)
+                if (tid + T * u < nwords) ss = sumsq_word(r[u], ss);
+            ss = group_sum(ss, red, grp);
+            const float inv = 1.0f / sqrtf(ss / (float)K + a.eps);
+#pragma unroll
+            for (int u = 0; u < kXRegWords; ++u) {
+                const int c = tid + T * u;
+                if constexpr (PRO == PRO_EMBED) {
+                    if (blockIdx.x == 0 && c < nwords) *reinterpret_cast<uint4 *>(a.resid_out + 8 * c) = r[u];
+                }
+                if (u < rounds) stage_word_tc(xt, sx8, c, nwords, c < nwords ? rmsnorm_word(r[u], gpre[u], inv) : zero);
+            }
+        } else {
+            float ss = 0.f;
+            for (int c = tid; c < nwords; c += T) ss = sumsq_word(*reinterpret_cast<const uint4 *>(src + 8 * c), ss);
+            issued();
+            ss = group_sum(ss, red, grp);
+            const float inv = 1.0f / sqrtf(ss / (float)K + a.eps);
+            for (int k = 0; k < rounds; ++k) {
+                const int c = tid + T * k;
+                uint4 x = zero;
+                if (c < nwords) {
+                    const uint4 rv = *reinterpret_cast<const uint4 *>(src + 8 * c);
+                    if constexpr (PRO == PRO_EMBED) {
+                        if (blockIdx.x == 0) *reinterpret_cast<uint4 *>(a.resid_out + 8 * c) = rv;
+                    }
+                    x = rmsnorm_word(rv, *reinterpret_cast<const uint4 *>(a.gamma + 8 * c), inv);
+                }
+                stage_word_tc(xt, sx8, c, nwords, x);
+            }
+        }
     }
 }
 
-template <int PRO, int EPI, int R, int KC>
+template <int PRO, int EPI, int R, int KC, bool DYN>
 __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvArgs a, const StreamGeom geo) {
     constexpr int PP = R / 2;               // row pairs per tile
     constexpr int WP = kConsumerWarps / PP;  // warps per row pair
+    static_assert(kWin == 8 && kConsumerWarps == 8 && (WP == 1 || WP == kConsumerWarps),
+                  "window flush: 8 tiles over 4-lane groups (one pair per warp) or over the 8 warps (one pair per tile)");
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full[kMaxStages];
     __shared__ __align__(8) uint64_t empty[kMaxStages];
+    __shared__ __align__(8) uint64_t xbar;  // the consumer warps have issued their loads of x
     __shared__ float red[32];
-    __shared__ float part[2][kConsumerWarps][2];
+    __shared__ float2 stash[kConsumerWarps][kWin][8];  // diagonal partial sums of a window
 
     const int K = a.K, wrow = K >> 1, groups = K >> 7, nb = tc_blocks(K);
     const int S = geo.stages;
     unsigned char *ring = smem;
     uint4 *xt = reinterpret_cast<uint4 *>(smem + (size_t)S * geo.stage_bytes);
     float *sx8 = reinterpret_cast<float *>(xt + (size_t)nb * 128);
-    const int t_begin = (int)(((long long)blockIdx.x * geo.tiles) / gridDim.x);
-    const int t_end = (int)(((long long)(blockIdx.x + 1) * geo.tiles) / gridDim.x);
-    const int n_tiles = t_end - t_begin;
+    __shared__ int stage_tile[kMaxStages];  // tile held by each stage; -1: no more tiles
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
+        mbar_init(&xbar, kConsumerWarps);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
+
+    // Tile order of this CTA. Static: a contiguous balanced range. Dynamic (a.sched given): the first
+    // kStaticTiles tiles c, c + G, ... then tiles claimed from a.sched[0] (offset by kStaticTiles * G)
+    // until they run out, so CTAs whose memory is served faster take more of the tail; the last CTA
+    // to run out resets both counters for the next launch.
+    const int G = gridDim.x, c = blockIdx.x;
+    const int t_begin = (int)(((long long)c * geo.tiles) / G);
+    const int t_end = (int)(((long long)(c + 1) * geo.tiles) / G);
+    const int n_tiles = t_end - t_begin;
+    constexpr bool dyn = DYN;  // the counter pair a.sched is given
+    auto static_tile = [&](int i) -> int {  // tile i of this CTA when known without the counter, else -2
+        if constexpr (!DYN) return t_begin + i < t_end ? t_begin + i : -1;
+        if (i < kStaticTiles) return c + i * G < geo.tiles ? c + i * G : -2;
+        return -2;
+    };
 
     unsigned long long best = 0ull;
     if (threadIdx.x < 32) {
         // ---------------- producer: weights do not depend on earlier kernels, so no dependency wait
         if (threadIdx.x == 0) {
             const uint64_t pol = evict_first_policy();
-            for (int i = 0; i < n_tiles; ++i) {
+            // geo.prex stages go out at once; the rest wait until x is requested, so the loads of x
+            // do not queue behind a whole ring of weight copies
+            const int prex = geo.prex < S ? geo.prex : S;
+            int claimed = -1;  // next counter value, requested one tile ahead so its latency overlaps a wait
+            if (dyn && kStaticTiles * G >= geo.tiles) claimed = geo.tiles;  // nothing left for the counter
+            // fixed ranges: exactly n_tiles stages, no end marker (the consumers know the count)
+            for (int i = 0; DYN || i < n_tiles; ++i) {
                 const int s = i % S, n = i / S;
+                int t = static_tile(i);
+                if (t == -2) {  // from the counter
+                    if (claimed < 0) claimed = kStaticTiles * G + (int)atomicAdd(&a.sched[0], 1u);
+                    t = claimed < geo.tiles ? claimed : -1;
+                    claimed = -1;
+                }
+                if (i == prex && !mbar_wait(&xbar, 0u)) {
+                    record_error(&g_device_error, 1);
+                    break;
+                }
                 if (n > 0 && !mbar_wait(&empty[s], (unsigned)((n - 1) & 1))) {
                     record_error(&g_device_error, 1);
                     break;
                 }
-                issue_tile<EPI, R>(a, t_begin + i, ring + (size_t)s * geo.stage_bytes, &full[s], pol);
-                if (i == (n_tiles < S ? n_tiles : S) - 1) {  // ring filled: spare DRAM time goes to the next kernel
+                if constexpr (DYN) {
+                    stage_tile[s] = t;
+                    if (t < 0) {
+                        mbar_arrive(&full[s]);  // the end marker: completes the phase without bytes
+                        break;
+                    }
+                }
+                issue_tile<EPI, R>(a, t, ring + (size_t)s * geo.stage_bytes, &full[s], pol);
+                if constexpr (DYN) {
+                    if (static_tile(i + 1) == -2 && claimed < 0)
+                        claimed = kStaticTiles * G + (int)atomicAdd(&a.sched[0], 1u);
+                }
+                if (i == S - 1) {  // ring filled: spare DRAM time goes to the next kernel
                     prefetch_share(a.pf_a, a.pf_a_bytes);
                     prefetch_share(a.pf_b, a.pf_b_bytes);
+                }
+            }
+            if constexpr (DYN) {
+                __threadfence();
+                if (atomicAdd(&a.sched[1], 1u) == (unsigned)G - 1) {  // every CTA has stopped claiming
+                    a.sched[0] = 0u;
+                    a.sched[1] = 0u;
+                    __threadfence();
                 }
             }
         }
     } else {
         // ---------------- consumers
         const NamedGroup<32, kConsumers> grp;
+        uint4 gpre[kXRegWords];
+#pragma unroll
+        for (int u = 0; u < kXRegWords; ++u) {
+            const int cw = grp.tid() + kConsumers * u;
+            gpre[u] = (PRO != PRO_PLAIN && cw < (K >> 3)) ? *reinterpret_cast<const uint4 *>(a.gamma + 8 * cw)
+                                                            : make_uint4(0u, 0u, 0u, 0u);
+        }
         grid_dep_wait();
         const EpiCta ecta = epi_cta<EPI>(a);  // issued before the staging so its latency overlaps it
-        stage_x_tc<PRO>(a, xt, sx8, red, grp);
+        // all of x in one round of loads when K is fixed (10 words per thread at K = 18944)
+        constexpr int LB = KC > 0 ? (KC / 8 + kConsumers - 1) / kConsumers : 4;
+        stage_x_tc<PRO, LB>(a, xt, sx8, red, grp, gpre, &xbar);
         grp.sync();
         grid_dep_launch();
         const int c_id = grp.tid(), warp = c_id >> 5, lane = c_id & 31;
         const int pr = warp / WP, wp = warp % WP;
         const int b0 = (wp * nb) / WP, b1 = ((wp + 1) * nb) / WP;
         const int tra = kPaired<EPI> ? pr : 2 * pr, trb = kPaired<EPI> ? pr + PP : 2 * pr + 1;
-        bool ok = true;
-        for (int i = 0; i < n_tiles; ++i) {
-            const int s = i % S, n = i / S, t = t_begin + i;
-            int ra0, na, rb0, nb_rows;
-            tile_rows<EPI, R>(a, t, ra0, na, rb0, nb_rows);
-            // epilogue inputs first: their global-memory latency overlaps the wait and the arithmetic
-            const int p = t * PP + pr;
-            int pa, pb;
-            pair_rows<EPI>(a, p, pa, pb);
-            const bool epi_lane = lane == 0 && wp == 0 && trb < na + nb_rows;
+        const int g8 = lane >> 2;
+        const bool diag = (lane & 3) == (g8 >> 1);  // the lane holding group g8's diagonal of the MMA
+        // the lane that finishes window tile fk: lane 4 fk of each warp (one pair per warp), or lane 0 of
+        // warp fk (one pair per tile, split over all warps)
+        const int fk = WP == 1 ? (lane >> 2) : warp;
+        const bool fin = WP == 1 ? (lane & 3) == 0 : lane == 0;
+        const int fpr = WP == 1 ? pr : 0;
+        const int ftrb = kPaired<EPI> ? fpr + PP : 2 * fpr + 1;
+        bool ok = true, more = true;
+        // Tiles go in windows of kWin: per tile only the dot products (the diagonal lanes park their
+        // partial sums in shared memory); the row sums and the epilogues of a whole window follow at
+        // its end, spread over lanes, so no reduction or epilogue latency sits between two tiles.
+        for (int i0 = 0; (DYN ? more : i0 < n_tiles) && ok; i0 += kWin) {
+            const int kn = DYN ? kWin : ((n_tiles - i0) < kWin ? (n_tiles - i0) : kWin);
+            // epilogue inputs: loaded now for tiles known in advance, else as the tile arrives
+            int ft = static_tile(i0 + fk), fp = 0, fpa = 0, fpb = 0;
+            bool flive = false;
             EpiIn ein = {0.f, 0.f, make_float2(0.f, 0.f), 0};
-            if (epi_lane) ein = epi_load<EPI>(a, p, pa, pb, ecta);
-            if (ok && !mbar_wait(&full[s], (unsigned)(n & 1))) {
-                record_error(&g_device_error, 1);
-                ok = false;
-            }
-            const bool live = ok && trb < na + nb_rows;
-            float tot_a = 0.f, tot_b = 0.f;
-            if (live) {
-                const unsigned char *st = ring + (size_t)s * geo.stage_bytes;
-                const uint16_t *sa = reinterpret_cast<const uint16_t *>(st + (size_t)R * wrow) + tra * groups;
-                const uint16_t *sb = reinterpret_cast<const uint16_t *>(st + (size_t)R * wrow) + trb * groups;
-                // K is a compile-time constant for the 7B shapes (KC > 0): offsets become immediates
-                const float2 tot = pair_dot<KC>(st, K, tra, trb, sa, sb, xt, sx8, b0, b1, lane);
-                tot_a = tot.x;
-                tot_b = tot.y;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
-            tot_a = warp_sum(tot_a);
-            tot_b = warp_sum(tot_b);
-            if constexpr (WP == 1) {
-                if (epi_lane && live) epilogue_in<EPI>(a, p, pa, pb, tot_a, tot_b, ein, ecta, best);
-            } else {
-                if (lane == 0) {
-                    part[i & 1][warp][0] = tot_a;
-                    part[i & 1][warp][1] = tot_b;
+            auto fin_setup = [&](int t) {
+                int ra0, na, rb0, nbr;
+                tile_rows<EPI, R>(a, t, ra0, na, rb0, nbr);
+                fp = t * PP + fpr;
+                pair_rows<EPI>(a, fp, fpa, fpb);
+                flive = fin && ftrb < na + nbr;
+                if (flive) ein = epi_load<EPI>(a, fp, fpa, fpb, ecta);
+            };
+            if (ft >= 0) fin_setup(ft);
+            int nw = 0;
+            for (int k = 0; k < kn; ++k) {
+                const int i = i0 + k, s = i % S, n = i / S;
+                ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (unsigned)(n & 1)));
+                if (!ok) {
+                    if (lane == 0) record_error(&g_device_error, 1);
+                    break;
                 }
-                grp.sync();
-                if (epi_lane && live) {
-                    float va = 0.f, vb = 0.f;
-                    for (int w = 0; w < WP; ++w) {
-                        va += part[i & 1][warp + w][0];
-                        vb += part[i & 1][warp + w][1];
+                int t = t_begin + i;  // fixed ranges: known without reading the stage
+                if constexpr (DYN) {
+                    t = *reinterpret_cast<volatile int *>(&stage_tile[s]);
+                    if (t < 0) {
+                        more = false;
+                        break;
                     }
-                    epilogue_in<EPI>(a, p, pa, pb, va, vb, ein, ecta, best);
                 }
+                if (k == fk && ft < 0) {
+                    ft = t;
+                    fin_setup(t);
+                }
+                int ra0, na, rb0, nb_rows;
+                tile_rows<EPI, R>(a, t, ra0, na, rb0, nb_rows);
+                float2 tot = make_float2(0.f, 0.f);
+                if (trb < na + nb_rows) {
+                    const unsigned char *st = ring + (size_t)s * geo.stage_bytes;
+                    const uint16_t *sa = reinterpret_cast<const uint16_t *>(st + (size_t)R * wrow) + tra * groups;
+                    const uint16_t *sb = reinterpret_cast<const uint16_t *>(st + (size_t)R * wrow) + trb * groups;
+                    // K is a compile-time constant for the 7B shapes (KC > 0): offsets become immediates
+                    tot = pair_dot<KC>(st, K, tra, trb, sa, sb, xt, sx8, b0, b1, lane);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
+                if (diag) stash[warp][k][g8] = tot;
+                nw = k + 1;
+            }
+            const bool mine = flive && ok && fk < nw;
+            if constexpr (WP == 1) {
+                __syncwarp();
+                const int q = lane & 3;
+                float2 v = make_float2(0.f, 0.f);
+                if (fk < nw) {
+                    const float2 u0 = stash[warp][fk][2 * q], u1 = stash[warp][fk][2 * q + 1];
+                    v = make_float2(u0.x + u1.x, u0.y + u1.y);
+                }
+                v.x += __shfl_xor_sync(0xffffffffu, v.x, 1);
+                v.y += __shfl_xor_sync(0xffffffffu, v.y, 1);
+                v.x += __shfl_xor_sync(0xffffffffu, v.x, 2);
+                v.y += __shfl_xor_sync(0xffffffffu, v.y, 2);
+                if (mine) epilogue_in<EPI>(a, fp, fpa, fpb, v.x, v.y, ein, ecta, best);
+                __syncwarp();  // the stash is rewritten by the next window
+            } else {
+                // every warp saw the same tiles (one pair per tile); a failed wait in one warp ends all
+                const bool all_ok = bar1_and(ok), all_more = bar1_and(more);
+                ok = all_ok;
+                more = all_more;
+                float2 v = make_float2(0.f, 0.f);
+                if (fk < nw) {  // 8 warps x 8 groups of partial sums for this tile's pair
+                    const float2 u0 = stash[lane >> 3][fk][lane & 7], u1 = stash[(lane >> 3) + 4][fk][lane & 7];
+                    v = make_float2(u0.x + u1.x, u0.y + u1.y);
+                }
+                v = warp_sum2(v);
+                if (mine) epilogue_in<EPI>(a, fp, fpa, fpb, v.x, v.y, ein, ecta, best);
+                grp.sync();
             }
         }
         if constexpr (EPI == EPI_ARGMAX) {
@@ -641,6 +850,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) gemv_tcb_kernel(const GemvA
 static bool g_stream_enabled = true;
 static int g_stream_smem_budget = 110 * 1024;  // two CTAs per SM
 static int g_stream_ctas_per_sm = 2;
+static int g_stream_prex = 1;
 
 void set_stream_options(int enabled, int smem_kb) {
     if (enabled >= 0) g_stream_enabled = enabled != 0;
@@ -648,8 +858,10 @@ void set_stream_options(int enabled, int smem_kb) {
 }
 
 void set_stream_ctas_per_sm(int n) { g_stream_ctas_per_sm = n; }
+void set_stream_prex(int n) { g_stream_prex = n; }
 
 bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp) {
+    g.prex = g_stream_prex;
     if (!g_stream_enabled || a.K % 512 != 0 || a.K > 32768 || a.N < 2) return false;
     if (unp == UNPACK_MMA && a.M > 1) {
         // batched tensor-core kernel: plain x, fp16/fp32 output, rows of up to 4096 weights
@@ -742,9 +954,9 @@ static int launch_stream_r(const GemvArgs &a, const StreamGeom &geo, cudaStream_
     }
 }
 
-template <int PRO, int EPI, int R, int KC>
-static int launch_tc_k(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
-    auto kern = gemv_tc_kernel<PRO, EPI, R, KC>;
+template <int PRO, int EPI, int R, int KC, bool DYN>
+static int launch_tc_kd(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
+    auto kern = gemv_tc_kernel<PRO, EPI, R, KC, DYN>;
     static int configured = -1;
     if (geo.smem > configured) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, geo.smem);
@@ -754,6 +966,16 @@ static int launch_tc_k(const GemvArgs &a, const StreamGeom &geo, cudaStream_t st
     if (g_dry_run) return I4_OK;
     return cuda_check(launch(kern, dim3(geo.grid), dim3(kStreamThreads), (size_t)geo.smem, stream, pdl, a, geo),
                       "tensor-core gemv launch");
+}
+
+// The shared-counter tile schedule (a.sched) is built for the residual and argmax epilogues (the down
+// projection and lm_head of the decode step, where it measured faster); other launches take fixed ranges.
+template <int PRO, int EPI, int R, int KC>
+static int launch_tc_k(const GemvArgs &a, const StreamGeom &geo, cudaStream_t stream, bool pdl) {
+    if constexpr (EPI == EPI_RESID || EPI == EPI_ARGMAX) {
+        if (a.sched) return launch_tc_kd<PRO, EPI, R, KC, true>(a, geo, stream, pdl);
+    }
+    return launch_tc_kd<PRO, EPI, R, KC, false>(a, geo, stream, pdl);
 }
 
 // rows of 3584 weights (16-row tiles) and 18944 weights (2-row tiles), the decoder's two row lengths, get

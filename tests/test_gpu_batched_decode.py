@@ -1,11 +1,15 @@
 """Batched decode (several sequences per step, one CUDA graph of library calls) vs the oracle.
 
-Three sequences with their own prompts and page-table rows over shared pools go
-through the prompt (teacher-forced, eager launches) and then 4 greedy steps (graph
-replays); every sequence's tokens must equal the oracle's greedy tokens for that
-sequence alone. The shape uses rows of 512-1024 weights so the batched
-tensor-core GEMV, the strided attention, the batched glue and the row argmax all
-run.
+3, 32 or 64 sequences with their own prompts and page-table rows over shared
+pools go through the prompt (teacher-forced, eager launches) and then 4 greedy
+steps (graph replays). Each sequence is compared with the oracle run on that
+sequence alone: its logits within 1e-2 normwise at every step while the two
+streams agree, and its tokens equal unless the oracle's top-2 gap at the parting
+step is within twice the GPU's own logit error there (a tie). The shape uses
+rows of 512-1024 weights. With 3 sequences the projections run on the batched
+tensor-core GEMV (mma.sync, up to 8 vectors); with 32 and 64 on the tcgen05 GEMM
+(split-K over the step's workspace). The strided attention, the batched glue and
+the row argmax run in every case.
 """
 import numpy as np
 import pytest
@@ -16,35 +20,55 @@ from int4_weight_only_02_b200 import synth
 pytestmark = pytest.mark.gpu
 
 
-def test_batched_decode_matches_oracle_per_sequence(i4lib, cuda):
+@pytest.mark.parametrize("B", [3, 32, 64])
+def test_batched_decode_matches_oracle_per_sequence(i4lib, cuda, B):
     import torch
     shape = synth.ModelShape(layers=2, hidden=512, inter=1024, n_q=4, n_kv=2, head_dim=128, vocab=1000, group=128,
                              page_size=16, max_ctx=64)
     layers = [synth.layer_weights(shape, i, 0) for i in range(shape.layers)]
     glob = synth.global_weights(shape, 0)
-    B, n_prompt, n_new = 3, 5, 4
+    n_prompt, n_new = 5, 4
     prompts = np.stack([synth.prompt_tokens(shape, n_prompt, seed=10 + b) for b in range(B)])
-    want = np.stack([oracle.DecoderOracle(shape, layers, glob, np.arange(shape.max_pages, dtype=np.int32))
-                     .generate(prompts[b], n_new)[0] for b in range(B)])
+    runs = [oracle.DecoderOracle(shape, layers, glob, np.arange(shape.max_pages, dtype=np.int32))
+            .generate(prompts[b], n_new) for b in range(B)]
+    want = np.stack([r[0] for r in runs])
+    want_logits = np.stack([r[1] for r in runs]).astype(np.float64)  # [B][n_new][vocab]
 
     rng = np.random.default_rng(7)
     tables = rng.permutation(B * shape.max_pages).astype(np.int32).reshape(B, shape.max_pages)
     model = i4lib.DeviceModel(shape, layers, glob, device=cuda)
     bd = i4lib.BatchedDecode(model, tables, num_pages=B * shape.max_pages)
+    assert (bd.gemm_ws is not None) == (B > 8)
     bd.reset(prompts[:, 0])
     for t in range(n_prompt):
         bd.step()
         if t + 1 < n_prompt:
             bd.tokens.copy_(torch.as_tensor(prompts[:, t + 1]))
     torch.cuda.synchronize()
-    got = [bd.tokens.cpu().numpy().copy()]
+    got, got_logits = [bd.tokens.cpu().numpy().copy()], [bd.logits.cpu().numpy().astype(np.float64)]
     bd.capture()
     for _ in range(n_new - 1):
         bd.replay()
         torch.cuda.synchronize()
         got.append(bd.tokens.cpu().numpy().copy())
-    got = np.stack(got, axis=1)
-    assert np.array_equal(got, want), (got, want)
+        got_logits.append(bd.logits.cpu().numpy().astype(np.float64))
+    got, got_logits = np.stack(got, axis=1), np.stack(got_logits, axis=1)
+    # Per sequence: while the streams agree the GPU saw the oracle's inputs, so its logits must be within
+    # the normwise tolerance of the small decoders; a token may differ only at a step whose oracle top-2
+    # gap is inside twice the GPU's own largest logit error there (a tie at this precision), and the
+    # stream is compared no further after it.
+    parted = []
+    for b in range(B):
+        for t in range(n_new):
+            err = np.abs(got_logits[b, t] - want_logits[b, t])
+            assert err.max() / np.abs(want_logits[b, t]).max() <= 1e-2, (b, t)
+            if got[b, t] != want[b, t]:
+                top = np.sort(want_logits[b, t])
+                assert top[-1] - top[-2] <= 2 * err.max(), (b, t, top[-1] - top[-2], err.max())
+                parted.append((b, t))
+                break
+    assert len(parted) <= max(1, B // 16), parted
+    print(f"B={B}: sequences parting at a tie: {parted}")
     assert np.array_equal(bd.pos.cpu().numpy(), np.full(B, n_prompt + n_new - 1))
     assert i4lib.device_error() == 0
 
