@@ -313,7 +313,8 @@ def teacher_forced(i4, model, shape, gold, torch):
             "oracle_gaps_below_0.1": int(np.sum(gaps < 0.1))}
 
 
-PROFILE_KERNELS = {"qkv": 0, "attention": 1, "o": 2, "gate_up": 3, "down": 4, "lm_head": 5, "token": -1}
+PROFILE_KERNELS = {"qkv": 0, "attention": 1, "o": 2, "gate_up": 3, "down": 4, "lm_head": 5, "token": -1,
+                   "gemm_gate_up_m512": -2}
 
 
 def run_profile_kernel(args):
@@ -336,8 +337,22 @@ def run_profile_kernel(args):
         i4.set_option("l2_prefetch", args.l2_prefetch)
     if args.persistent is not None:
         i4.set_option("persistent", args.persistent)
-    shape = synth.ModelShape(layers=1)
     dev = torch.device("cuda", 0)
+    if PROFILE_KERNELS[args.profile_kernel] == -2:  # prompt-prefill gate/up GEMM (tcgen05): M = 512 rows
+        shape = synth.QWEN7B
+        lw = synth.layer_weights(shape, 0, 0)
+        w, sc = (i4.runtime.to_device(lw[k], dev) for k in ("w_gu", "s_gu"))
+        x = (torch.randn(512, shape.hidden, device=dev) * 0.5).half()
+        n_out = 2 * shape.inter
+        y = torch.empty(512, n_out, device=dev, dtype=torch.float16)
+        ws = torch.zeros(max(i4.int4_gemm_ws_bytes(512, n_out, shape.hidden), 256), dtype=torch.uint8, device=dev)
+        for _ in range(args.launches):
+            i4.int4_gemm(w, sc, x, y=y, ws=ws)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_kernel": args.profile_kernel, "launches": args.launches,
+                          "M": 512, "N": n_out, "K": shape.hidden, "device_error": i4.device_error()}))
+        return 0
+    shape = synth.ModelShape(layers=1)
     layers = [synth.layer_weights(synth.QWEN7B, 0, 0)]
     glob = synth.global_weights(shape, 0)
     model = i4.DeviceModel(shape, layers, glob, device=dev)
