@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     record_error(&g_gemm_error, 1);
                     break;
                 }
-                if (gemm_aborted()) break;
+                if ((c & 15) == 15 && gemm_aborted()) break;  // a global read: not on every chunk's path
                 const int kc = c_begin + c;
                 mbar_expect_tx(&raw_full[s], kGRaw + (unsigned)BN * 128u);
                 tma_load_2d(stage_raw(s), &tm_w, kc * (kGBK / 2), n0, &raw_full[s]);
