@@ -100,9 +100,10 @@ def test_embed_gather_and_argmax_rows(i4lib, cuda):
 @pytest.mark.parametrize("inter,n_prompt,graph", [(1024, 24, True), (1024, 40, False), (12288, 40, True)])
 def test_chunked_prefill_matches_oracle(i4lib, cuda, inter, n_prompt, graph):
     """Prefill of one sequence 8 positions per step (rows = consecutive positions over one page-table
-    row): the first generated token and the last position's logits equal the oracle's. Prompts of 3
-    and 5 chunks cross partially filled pages; eager and graph steps; intermediate 12288 sends the
-    down projection through the split 4-vector calls."""
+    row): the first generated token and the last position's logits equal the oracle's, and two decode
+    steps continued from the prefilled pages (continue_state) give the oracle's next tokens in every
+    row. Prompts of 3 and 5 chunks cross partially filled pages; eager and graph steps; intermediate
+    12288 sends the down projection through the split 4-vector calls."""
     import torch
     shape = synth.ModelShape(layers=2, hidden=512, inter=inter, n_q=4, n_kv=2, head_dim=128, vocab=1000,
                              group=128, page_size=16, max_ctx=64)
@@ -122,6 +123,16 @@ def test_chunked_prefill_matches_oracle(i4lib, cuda, inter, n_prompt, graph):
     assert got == want
     got_logits = bd.logits[7].cpu().numpy().astype(np.float64)
     assert np.max(np.abs(got_logits - want_logits)) / np.max(np.abs(want_logits)) <= 1e-2
+    # decode continues from the prefilled pages: every row then steps the same sequence
+    want_cont = oracle.DecoderOracle(shape, layers, glob, table).generate(prompt, 3)[0]
+    assert want_cont[0] == want
+    bd.continue_state(n_prompt, got)
+    import torch
+    for step in (1, 2):
+        bd.step()
+        torch.cuda.synchronize()
+        toks = bd.tokens.cpu().numpy()
+        assert np.all(toks == want_cont[step]), (step, toks, want_cont)
     assert i4lib.device_error() == 0
 
 
