@@ -21,11 +21,16 @@ from helpers import FLIP_RATE, LOGIT_NOISE_MAX, TIE_GAP
 LOGIT_NOISE_ONE_ULP = 0.075  # largest single-logit change from one ulp in one input element (measured 0.073)
 
 
-@pytest.mark.slow
-def test_one_ulp_input_change_moves_logits_by_hundredths():
+@pytest.fixture(scope="module")
+def qwen7b():
+    """The 28-layer random-init 7B-shape decoder (seed 0), generated once for both tests."""
     shape = synth.QWEN7B
-    layers = [synth.layer_weights(shape, i, 0) for i in range(shape.layers)]
-    glob = synth.global_weights(shape, 0)
+    return shape, [synth.layer_weights(shape, i, 0) for i in range(shape.layers)], synth.global_weights(shape, 0)
+
+
+@pytest.mark.slow
+def test_one_ulp_input_change_moves_logits_by_hundredths(qwen7b):
+    shape, layers, glob = qwen7b
     tok = 12345
     ref_traces = []
     ref = oracle.DecoderOracle(shape, layers, glob, synth.page_table(shape, 0)).forward([tok], 0, ref_traces)[0]
@@ -57,7 +62,7 @@ def _flipping_f16(rng, rate):
 
 
 @pytest.mark.slow
-def test_measured_flip_rate_sets_the_greedy_tie_bound(monkeypatch):
+def test_measured_flip_rate_sets_the_greedy_tie_bound(monkeypatch, qwen7b):
     """Noise model of fp32-vs-fp64 accumulation: FLIP_RATE (the largest independent fp16
     mismatch rate measured per tensor on the GPU, 1.7 %) of every stored fp16 tensor one ulp off.
 
@@ -65,9 +70,7 @@ def test_measured_flip_rate_sets_the_greedy_tie_bound(monkeypatch):
     RMS; three standard deviations of a top-2 gap difference must stay within
     the tie bound the GPU decode test uses, and the largest logit change within
     the first-step noise ceiling."""
-    shape = synth.QWEN7B
-    layers = [synth.layer_weights(shape, i, 0) for i in range(shape.layers)]
-    glob = synth.global_weights(shape, 0)
+    shape, layers, glob = qwen7b
     prompt = synth.prompt_tokens(shape, 64, 7)
     ref = oracle.DecoderOracle(shape, layers, glob, synth.page_table(shape, 0)).forward(prompt, 0)[0]
     noisy = _flipping_f16(np.random.default_rng(200), FLIP_RATE)
