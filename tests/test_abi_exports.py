@@ -64,6 +64,14 @@ def test_host_validation_without_gpu(i4lib):
     assert L.paged_gqa_decode_ws_bytes(1, 28, 4, 64, 16, 256) == 0
     assert L.decode_step_graph_replay(None, None) == i4lib.I4_EINVAL
     assert L.i4_set_option(b"nonsense", 1) == i4lib.I4_EINVAL
+    # option ranges (host-side settings, no GPU involved); defaults restored afterwards
+    assert L.i4_set_option(b"gemv_prex", 9) == i4lib.I4_EINVAL
+    assert L.i4_set_option(b"gemv_prex", -1) == i4lib.I4_EINVAL
+    assert L.i4_set_option(b"gemv_prex", 2) == i4lib.I4_OK
+    assert L.i4_set_option(b"gemv_prex", 1) == i4lib.I4_OK
+    assert L.i4_set_option(b"gemv_ctas_per_sm", 3) == i4lib.I4_EINVAL
+    assert L.i4_set_option(b"stream_smem_kb", 8) == i4lib.I4_EINVAL
+    assert L.i4_set_option(b"unpack", 9) == i4lib.I4_EINVAL
 
 
 def test_batched_decode_entries_validate_without_gpu(i4lib):

@@ -164,3 +164,24 @@ def test_batched_tensor_core_exact_arithmetic(i4lib, cuda):
     for i in range(m):
         ref = oracle.int4_gemv(w, s, x[i], None)
         assert np.array_equal(got[i].view(np.uint16), ref.view(np.uint16)), i
+
+
+@pytest.mark.parametrize("n,k", [(37888, 3584), (3584, 18944)])
+def test_weight_stage_holdback_keeps_bits(i4lib, cuda, n, k):
+    """The number of weight stages copied before x is requested (option gemv_prex) changes only when
+    copies start: the outputs are bit-identical for 0, 1 (default) and 3 stages."""
+    import torch
+    w, s, x, _ = synth.gemv_case(n, k, seed=11)
+    args = [dev(a, cuda) for a in (w, s, x)]
+    outs = []
+    try:
+        for prex in (0, 1, 3):
+            i4lib.set_option("gemv_prex", prex)
+            outs.append(i4lib.int4_gemv(*args).cpu().numpy())
+    finally:
+        i4lib.set_option("gemv_prex", 1)
+    torch.cuda.synchronize()
+    assert np.array_equal(outs[0].view(np.uint16), outs[1].view(np.uint16))
+    assert np.array_equal(outs[2].view(np.uint16), outs[1].view(np.uint16))
+    assert normwise_err(outs[1][0], oracle.int4_gemv(w, s, x[0])) <= TOL
+    assert i4lib.device_error() == 0
