@@ -365,6 +365,10 @@ I4_API int decode_step_buffer_copy(i4_graph *g, int which, void *dev, size_t byt
  *            (M == 1, K % 512 == 0, 16-byte aligned w and scales), default 1;
  *   "stream_smem_kb" 32..227: shared memory budget of that kernel's ring;
  *   "gemv_ctas_per_sm" 1/2 (default 2): CTAs per SM of the pipelined GEMV grids;
+ *   "test_stall" 0/1 (default 0): for tests of the bounded waits only: the
+ *            tensor-core GEMV's producer skips its first copy, its consumers'
+ *            wait and then its own run out (~2 s each), the launch records
+ *            device error 1 (i4_device_error) and returns; never set it in use;
  *   "gemv_prex" 0..8 (default 1): weight stages the tensor-core GEMV copies
  *            before its loads of x are issued (the rest follow them, so x does
  *            not queue behind a full ring of weight copies);

@@ -539,6 +539,10 @@ extern "C" int i4_set_option(const char *name, int value) {
         g_l2_prefetch = value != 0;
         return I4_OK;
     }
+    if (n == "test_stall") {
+        set_test_stall(value != 0);
+        return I4_OK;
+    }
     if (n == "gemv_prex") {
         if (value < 0 || value > 8) return fail(I4_EINVAL, "gemv_prex must be in [0, 8]");
         set_stream_prex(value);

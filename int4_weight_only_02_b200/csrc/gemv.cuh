@@ -65,6 +65,7 @@ struct StreamGeom {
     int tiles, tiles_per_cta, grid;
     int smem;           // dynamic shared memory bytes
     int prex;           // tensor-core consumer: stages copied before the loads of x are issued
+    int test_stall;     // tests of the bounded waits: the producer skips its first copy (see set_test_stall)
 };
 // False when the shape or alignment does not fit the streaming kernel.
 bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp);
@@ -73,6 +74,10 @@ int launch_gemv_stream(int pro, int epi, const GemvArgs &a, const StreamGeom &ge
 void set_stream_options(int enabled, int smem_kb);
 void set_stream_ctas_per_sm(int n);
 void set_stream_prex(int n);
+// Test of the bounded waits: while set, the tensor-core GEMV's producer never copies its first tile, so the
+// consumers' wait for it and then the producer's wait for a free stage run out (~2 s each) and the kernel
+// records device error 1 and returns; no fault, the context stays usable.
+void set_test_stall(int on);
 // unp < 0 selects the library default; max_ctas <= 0 means no cap.
 int launch_gemv(int pro, int epi, const GemvArgs &a, cudaStream_t stream, bool pdl, int unp, int max_ctas);
 

@@ -546,6 +546,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2) gemv_tc_kernel(const GemvAr
                         break;
                     }
                 }
+                if (geo.test_stall && i == 0) continue;  // the bounded-wait test: stage 0 never fills
                 issue_tile<EPI, R>(a, t, ring + (size_t)s * geo.stage_bytes, &full[s], pol);
                 if constexpr (DYN) {
                     if (static_tile(i + 1) == -2 && claimed < 0)
@@ -851,6 +852,7 @@ static bool g_stream_enabled = true;
 static int g_stream_smem_budget = 110 * 1024;  // two CTAs per SM
 static int g_stream_ctas_per_sm = 2;
 static int g_stream_prex = 1;
+static int g_test_stall = 0;
 
 void set_stream_options(int enabled, int smem_kb) {
     if (enabled >= 0) g_stream_enabled = enabled != 0;
@@ -859,9 +861,11 @@ void set_stream_options(int enabled, int smem_kb) {
 
 void set_stream_ctas_per_sm(int n) { g_stream_ctas_per_sm = n; }
 void set_stream_prex(int n) { g_stream_prex = n; }
+void set_test_stall(int on) { g_test_stall = on; }
 
 bool stream_geometry(int epi, const GemvArgs &a, StreamGeom &g, int unp) {
     g.prex = g_stream_prex;
+    g.test_stall = g_test_stall;
     if (!g_stream_enabled || a.K % 512 != 0 || a.K > 32768 || a.N < 2) return false;
     if (unp == UNPACK_MMA && a.M > 1) {
         // batched tensor-core kernel: plain x, fp16/fp32 output, rows of up to 4096 weights

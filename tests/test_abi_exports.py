@@ -72,6 +72,7 @@ def test_host_validation_without_gpu(i4lib):
     assert L.i4_set_option(b"gemv_ctas_per_sm", 3) == i4lib.I4_EINVAL
     assert L.i4_set_option(b"stream_smem_kb", 8) == i4lib.I4_EINVAL
     assert L.i4_set_option(b"unpack", 9) == i4lib.I4_EINVAL
+    assert L.i4_set_option(b"test_stall", 0) == i4lib.I4_OK
 
 
 def test_batched_decode_entries_validate_without_gpu(i4lib):

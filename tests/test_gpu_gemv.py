@@ -185,3 +185,25 @@ def test_weight_stage_holdback_keeps_bits(i4lib, cuda, n, k):
     assert np.array_equal(outs[2].view(np.uint16), outs[1].view(np.uint16))
     assert normwise_err(outs[1][0], oracle.int4_gemv(w, s, x[0])) <= TOL
     assert i4lib.device_error() == 0
+
+
+def test_bounded_wait_reports_and_the_context_recovers(i4lib, cuda):
+    """Failure detection without a fault: with the test-only stall the producer never copies its first
+    tile, so the consumers' wait for it and the producer's wait for a free stage run out (~2 s each).
+    The launch returns, the host reads device error 1, and the next call on the same context is
+    correct."""
+    import torch
+    w, s, x, b = synth.gemv_case(4608, 3584, seed=12, bias=True)
+    args = [dev(a, cuda) for a in (w, s, x)]
+    bias = dev(b, cuda)
+    assert i4lib.device_error() == 0
+    i4lib.set_option("test_stall", 1)
+    try:
+        i4lib.int4_gemv(*args, bias=bias)
+        torch.cuda.synchronize()
+    finally:
+        i4lib.set_option("test_stall", 0)
+    assert i4lib.device_error() == 1  # read and cleared
+    got = i4lib.int4_gemv(*args, bias=bias).cpu().numpy()[0]
+    assert normwise_err(got, oracle.int4_gemv(w, s, x[0], b)) <= TOL
+    assert i4lib.device_error() == 0
