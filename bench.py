@@ -941,9 +941,12 @@ def main():
     eager_ms = e0.elapsed_time(e1) / max(args.eager_steps, 1)
 
     # dominant kernel alone: RMSNorm + gate/up GEMV + SiLU of each layer (70 MB each, L2-cold)
-    def time_kernel(index_fn, reps=3):
+    spreads = {}
+
+    def time_kernel(index_fn, reps=10, name=None):
         """Mean device time of one launch: the kernel of every layer captured back to back in one
-        CUDA graph, replayed `reps` times between two events on the launching stream."""
+        CUDA graph, each of `reps` replays timed between two events on the launching stream; the
+        per-launch minimum and maximum over the replays go to spreads[name]."""
         side = torch.cuda.Stream()
         cg = torch.cuda.CUDAGraph()
         torch.cuda.synchronize()
@@ -954,29 +957,32 @@ def main():
         torch.cuda.synchronize()
         cg.replay()
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        ev[0].record(stream)
+        for r in range(reps):
             cg.replay()
-        e1.record(stream)
+            ev[r + 1].record(stream)
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / (reps * shape.layers)
+        per = [ev[r].elapsed_time(ev[r + 1]) / shape.layers for r in range(reps)]
+        if name:
+            spreads[name] = (min(per), max(per))
+        return ev[0].elapsed_time(ev[reps]) / (reps * shape.layers)
 
     h, inter = shape.hidden, shape.inter
     gu_bytes = 2 * inter * (h // 2) + 2 * inter * (h // 128) * 2 + 2 * h * 2 + inter * 2
-    gu_ms = time_kernel(lambda li: 5 * li + 3)
+    gu_ms = time_kernel(lambda li: 5 * li + 3, name="gate_up")
     down_bytes = h * (inter // 2) + h * (inter // 128) * 2 + inter * 2 + 2 * h * 2
-    down_ms = time_kernel(lambda li: 5 * li + 4)
+    down_ms = time_kernel(lambda li: 5 * li + 4, name="down")
     qkv_rows = shape.qkv_rows
     qkv_bytes = qkv_rows * (h // 2) + qkv_rows * (h // 128) * 2 + 2 * qkv_rows * 2 + 2 * h * 2
-    qkv_ms = time_kernel(lambda li: 5 * li + 0)
+    qkv_ms = time_kernel(lambda li: 5 * li + 0, name="qkv")
     o_bytes = h * (h // 2) + h * (h // 128) * 2 + h * 2 + 2 * h * 2
-    o_ms = time_kernel(lambda li: 5 * li + 2)
-    attn_ms = time_kernel(lambda li: 5 * li + 1)
+    o_ms = time_kernel(lambda li: 5 * li + 2, name="o")
+    attn_ms = time_kernel(lambda li: 5 * li + 1, name="attention")
     # lm_head: the last kernel of the step, launched 28 times (it also advances the sequence state,
     # which nothing reads afterwards)
     lm_bytes = shape.vocab * (h // 2) + shape.vocab * (h // 128) * 2 + shape.vocab * 4 + 2 * h * 2
-    lm_ms = time_kernel(lambda li: graph.phase_count - 1)
+    lm_ms = time_kernel(lambda li: graph.phase_count - 1, name="lm_head")
     torch.cuda.synchronize()
     # restore a consistent residual/KV state is not needed afterwards: nothing else runs
 
@@ -1015,7 +1021,9 @@ def main():
                    "kernels_per_step": n_k, "status": status},
         "roofline": roofline,
         "persistent_step": graph.persistent,
-        # each phase launched alone (its own launch, stream start-up and drain): diagnostics only
+        # each phase launched alone (its own launch, stream start-up and drain): diagnostics only; mean
+        # over 10 graph replays of the 28 launches, with the per-launch min/max over the replays
+        "phase_launches_spread_us": {k: [round(a * 1e3, 2), round(b * 1e3, 2)] for k, (a, b) in spreads.items()},
         "phase_launches": {
             "qkv": {"us": round(qkv_ms * 1e3, 2), "GBs": round(qkv_bytes / (qkv_ms * 1e-3) / 1e9, 1)},
             "o": {"us": round(o_ms * 1e3, 2), "GBs": round(o_bytes / (o_ms * 1e-3) / 1e9, 1)},
